@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the SVDQuant W4A4 NVFP4 linear layer on B200.
+
+Workload: the fused-QKV projection of a DiT block at 1024x1024 (M = 4608
+tokens = 4096 image + 512 text, K = 3072, N = 9216, rank 32, NVFP4 group 16),
+seeded synthetic inputs (synth/). One step = the whole hot path over one batch:
+svdq_quantize_act (smoothing + NVFP4 quantisation + x_hat L1) followed by
+svdq_w4a4_linear (block-scaled FP4 GEMM + P L2 + bias). The weight pack is
+offline and not timed.
+
+Metric: TFLOPS counted as 2 M N K per step (the low-rank flops are not
+counted), and that value as a fraction of the dense FP4 peak.
+
+Timing: W untimed warm-up steps, then K timed steps. Before every step a
+512 MiB buffer is written (L2 is 126 MB) outside the step's events, so each
+step starts with a cold L2. Steps are timed with CUDA events on the launching
+stream; the timed loop is bracketed by a barrier and a device synchronise on
+both sides; with several GPUs every rank runs its own replica (independent
+batches: weak scaling, no collective on the data path) and the per-step time
+is the maximum over ranks.
+
+``--impl reference`` times the CPU oracle (the only reference implementation
+of this path) on a bounded row sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "c3_qkv_nvfp4"
+METRIC = "SVDQ W4A4-NVFP4 linear TFLOPS, % dense FP4 peak (M4608 K3072 N9216 r32)"
+FP4_DENSE_SPEC_TFLOPS = 9000.0
+NOMINAL_FP4_OVER_BF16 = 4.0     # 9 PF / 2.25 PF dense
+L2_FLUSH_BYTES = 512 << 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+# --------------------------------------------------------------------------- CUDA arm
+def run_cuda(args):
+    import bit_w4a4_quantized_nvfp4_b200 as svdq
+
+    world, rank, local = dist_setup(args.gpus)
+    svdq.load()
+    c = synth.CONFIGS[WORKLOAD]
+    M, K, N, r = c["M"], c["K"], c["N"], c["r"]
+    d = synth.config_layer(WORKLOAD)
+    W = torch.from_numpy(d["W"]).cuda()
+    lam = torch.from_numpy(d["lam"]).cuda()
+    L1, L2, b = bf16_dev(d["L1"]), bf16_dev(d["L2"]), bf16_dev(d["b"])
+    x = bf16_dev(d["x"])
+    pw = svdq.pack_weight("nvfp4", W, lam, L1, L2)
+    del W
+    stream = torch.cuda.current_stream()
+    qa = svdq.quantize_act(x, pw, L1)
+    y = svdq.w4a4_linear(qa, pw, b)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    svdq.device_error()
+
+    def step():
+        svdq.quantize_act(x, pw, L1, out=qa)
+        svdq.w4a4_linear(qa, pw, b, out=y)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    K_steps = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K_steps):
+        flush.zero_()
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        svdq.quantize_act(x, pw, L1, out=qa)
+        e1.record(stream)
+        svdq.w4a4_linear(qa, pw, b, out=y)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    svdq.device_error()
+
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
+    k1_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    k2_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    ms = max_over_ranks(world, statistics.mean(step_ms))
+    k1 = max_over_ranks(world, statistics.mean(k1_ms))
+    k2 = max_over_ranks(world, statistics.mean(k2_ms))
+    flops = 2.0 * M * N * K
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers
+    xh = torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16)).pin_memory()
+    yh = torch.empty((M, N), dtype=torch.int16).pin_memory()
+    xd = torch.empty((M, K), dtype=torch.int16, device="cuda")
+    e2e_steps = max(3, min(20, K_steps))
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        svdq.svdq_linear(xd.view(torch.bfloat16), pw, L1, b)
+    torch.cuda.synchronize()
+    barrier(world)
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record(stream)
+    for _ in range(e2e_steps):
+        xd.copy_(xh, non_blocking=True)
+        yo = svdq.svdq_linear(xd.view(torch.bfloat16), pw, L1, b)
+        yh.copy_(yo.view(torch.int16), non_blocking=True)
+    ee.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, es.elapsed_time(ee) / e2e_steps)
+    barrier(world)
+
+    P = peaks()
+    fp4_peak = P["bf16"] * NOMINAL_FP4_OVER_BF16
+    k2_tflops = flops / (k2 * 1e-3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": {"workload": f"svdq_w4a4 nvfp4 fused-QKV projection M{M} K{K} N{N} r{r} (seeded DiT-shaped "
+                               "inputs, 0.5% outlier channels x30)",
+                   "M": M, "K": K, "N": N, "r": r, "group": 16,
+                   "l2": "flushed before every timed step (512 MiB write, outside the step's events)",
+                   "parallelism": f"{world} independent replicas (weak scaling, no collective)"},
+        "pct_dense_fp4_peak_spec": round(100.0 * value / world / FP4_DENSE_SPEC_TFLOPS, 2),
+        "kernels_ms": {"quantize_act": round(k1, 5), "w4a4_gemm": round(k2, 5)},
+        "roofline": {"kernel": "w4a4_gemm (tcgen05 mxf4nvf4)", "bound": "tensor",
+                     "achieved": round(k2_tflops, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(k2_tflops / fp4_peak, 4),
+                     "peak_source": f"{P['source']} bf16 burst {P['bf16']} x nominal fp4/bf16 ratio 4",
+                     "traffic": None},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "gpu_launches": 2 * K_steps,
+        "wall_s_timed_region": round(wall, 4),
+    }
+    if clk:
+        out["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(d, rows=args.cpu_rows)
+    if rank == 0 and not args.no_awq:
+        out["awq_gemv"] = bench_awq(svdq, P)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def bench_awq(svdq, P):
+    """AWQ W4A16 GEMV (M = 1, K 3072, N 18432): HBM-bound; weights rotate over
+    copies totalling > 3x L2 so every launch streams from HBM."""
+    c = synth.CONFIGS["c2_awq_gemv"]
+    K, N = c["K"], c["N"]
+    d = synth.awq_inputs(c["seed"], 1, K, N)
+    w0 = svdq.awq_pack_weight(torch.from_numpy(d["W"]).cuda())
+    copies = []
+    for _ in range(12):  # 12 x 31.9 MB = 383 MB
+        copies.append(svdq.AwqWeight(K, N, w0.q.clone(), w0.scales.clone(), w0.zeros.clone()))
+    x = bf16_dev(d["x"])
+    y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    for w in copies:
+        svdq.awq_w4a16_linear(x, w, out=y)
+    torch.cuda.synchronize()
+    reps = 20
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        for w in copies:
+            svdq.awq_w4a16_linear(x, w, out=y)
+    e.record()
+    torch.cuda.synchronize()
+    us = s.elapsed_time(e) * 1e3 / (reps * len(copies))
+    byts = N * K // 2 + 2 * 2 * N * (K // 64) + K * 2 + N * 2
+    gbs = byts / (us * 1e-6) / 1e9
+    return {"M": 1, "K": K, "N": N, "us_per_launch": round(us, 3), "algorithmic_bytes": byts,
+            "achieved_gbs": round(gbs, 1), "peak_gbs": P["hbm_gbs"], "frac": round(gbs / P["hbm_gbs"], 4)}
+
+
+# --------------------------------------------------------------------------- oracle
+def cpu_baseline(d, rows: int, tag="oracle"):
+    import oracle
+
+    c = synth.CONFIGS[WORKLOAD]
+    K, N = c["K"], c["N"]
+    w = oracle.pack_weight("nvfp4", d["W"], d["lam"], d["L1"], d["L2"])
+    x = d["x"][:rows]
+    t0 = time.perf_counter()
+    a = oracle.quantize_act("nvfp4", x, w["inv_lam"], 1.0, d["L1"])
+    oracle.linear("nvfp4", a, w, 1.0, d["L2"], d["b"])
+    dt = time.perf_counter() - t0
+    return {"value": round(2.0 * rows * N * K / dt / 1e12, 6), "unit": "TFLOPS", "cores": oracle.threads(),
+            "kind": tag, "sample": f"first {rows} of {c['M']} rows of the workload (quantize_act + linear, "
+                                    "float64 accumulation); weight pack untimed", "seconds": round(dt, 3)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+
+    c = synth.CONFIGS[WORKLOAD]
+    M, K, N, r = c["M"], c["K"], c["N"], c["r"]
+    d = synth.config_layer(WORKLOAD)
+    w = oracle.pack_weight("nvfp4", d["W"], d["lam"], d["L1"], d["L2"])
+    rows = args.ref_rows
+    times = []
+    for i in range(args.warmup + args.steps):
+        lo = (i * rows) % M
+        x = d["x"][lo:lo + rows]
+        t0 = time.perf_counter()
+        a = oracle.quantize_act("nvfp4", x, w["inv_lam"], 1.0, d["L1"])
+        oracle.linear("nvfp4", a, w, 1.0, d["L2"], d["b"])
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    s = statistics.mean(times)
+    value = 2.0 * rows * N * K / s / 1e12
+    sample = f"{rows} rows per step of the M{M} K{K} N{N} r{r} workload (CPU oracle, float64 accumulation)"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"svdq_w4a4 nvfp4 fused-QKV projection M{M} K{K} N{N} r{r}", "M": M, "K": K,
+                   "N": N, "r": r, "rows_per_step": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-awq", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

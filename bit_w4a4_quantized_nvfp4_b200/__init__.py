@@ -1,0 +1,275 @@
+"""B200 (sm_100a) SVDQuant W4A4 and AWQ W4A16 linear layers.
+
+A thin ctypes binding over ``libsvdq.so`` (C ABI in ``include/svdq.h``).
+Every function here only marshals arguments: torch tensors provide device
+memory and the current CUDA stream, and every step of the layer runs in the
+library's kernels. There is no CPU fallback: importing works without a GPU,
+but calling an entry point without the built library raises.
+
+The layer (blog "Introducing Nunchaku 4-bit inference in Diffusers", section
+"Background: SVDQuant and Nunchaku"):
+    y = Q4(x_hat) . Q4(R) + (x_hat L1) L2 + b,  x_hat = bf16(x / lambda),
+    R = diag(lambda) W - L1 L2,
+with svdq_w4a4 NVFP4 (group 16) or INT4 (group 64) and awq_w4a16 INT4
+(group 64) (Diffusers "Nunchaku Lite" page, table "Supported quantization
+types").
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import enum
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "NVFP4", "INT4", "Status", "SvdqError", "PackedWeight", "QuantAct", "AwqWeight",
+    "library_path", "load", "scale_bytes", "pack_weight", "quantize_act", "w4a4_linear",
+    "svdq_linear", "awq_pack_weight", "awq_w4a16_linear", "device_error", "set_wait_limit_ns",
+    "probe_convert", "probe_wait_timeout", "debug_force_arch",
+]
+
+NVFP4, INT4 = 0, 1
+_OUT = {"bf16": 0, "f32": 1, "i32_groups": 2}
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+class Status(enum.IntEnum):
+    OK = 0
+    INVALID_ARG = 1
+    SHAPE = 2
+    ALIGN = 3
+    UNSUPPORTED_ARCH = 4
+    CUDA = 5
+    TIMEOUT = 6
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = Status(status)
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libsvdq.so")
+
+
+# name -> (restype, argtypes)
+_P, _I, _F, _U64, _I64 = C.c_void_p, C.c_int, C.c_float, C.c_ulonglong, C.c_longlong
+SIGNATURES = {
+    "svdq_status_str": (C.c_char_p, [_I]),
+    "svdq_scale_bytes": (C.c_size_t, [_I, _I, _I]),
+    "svdq_lr_up_elems": (C.c_size_t, [_I, _I, _I]),
+    "svdq_pack_weight": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P]),
+    "svdq_quantize_act": (_I, [_I, _I, _I, _I, _P, _P, _F, _P, _P, _P, _P, _P]),
+    "svdq_w4a4_linear": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "awq_pack_weight": (_I, [_I, _I, _P, _P, _P, _P, _P]),
+    "awq_w4a16_linear": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "svdq_device_error": (_I, [_P]),
+    "svdq_set_wait_limit_ns": (None, [_U64]),
+    "svdq_probe_convert": (_I, [_P, _I64, _P, _P, _P, _P]),
+    "svdq_probe_wait_timeout": (_I, [_U64, _P]),
+    "svdq_debug_force_arch": (None, [_I, _I]),
+}
+
+
+def load():
+    """Load ``libsvdq.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m bit_w4a4_quantized_nvfp4_b200.build` "
+                "(nvcc, sm_100a); this package has no fallback implementation")
+        L = C.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise SvdqError(fn, status, load().svdq_status_str(status).decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _prec(p) -> int:
+    if isinstance(p, str):
+        return {"nvfp4": NVFP4, "int4": INT4}[p]
+    return int(p)
+
+
+def scale_bytes(prec, rows: int, K: int) -> int:
+    return int(load().svdq_scale_bytes(_prec(prec), rows, K))
+
+
+@dataclass
+class PackedWeight:
+    prec: int
+    K: int
+    N: int
+    r: int
+    codes: torch.Tensor          # uint8 [N, K/2]
+    scales: torch.Tensor         # uint8 (tiled e4m3 bytes or bf16 pairs)
+    tensor_scale: torch.Tensor   # float32 [2] = {s_tw, s_tx}
+    inv_lambda: torch.Tensor     # float32 [K]
+    lr_up: Optional[torch.Tensor]  # bf16 [N, 2r] (NVFP4) or [N, r] (INT4)
+    act_tensor_scale: float
+
+
+@dataclass
+class QuantAct:
+    prec: int
+    M: int
+    K: int
+    r: int
+    codes: torch.Tensor    # uint8 [M, K/2]
+    scales: torch.Tensor   # uint8 bytes
+    P: Optional[torch.Tensor]  # bf16 [M, r]
+
+
+def pack_weight(prec, W: torch.Tensor, lam: torch.Tensor, L1: Optional[torch.Tensor],
+                L2: Optional[torch.Tensor], act_tensor_scale: float = 1.0, stream=None) -> PackedWeight:
+    """svdq_pack_weight: W fp32 [K, N], lam fp32 [K], L1 bf16 [K, r], L2 bf16 [r, N]."""
+    p = _prec(prec)
+    K, N = W.shape
+    r = 0 if L1 is None else L1.shape[1]
+    dev = W.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(max(scale_bytes(p, N, K), 16), dtype=torch.uint8, device=dev)
+    ts = torch.empty(4, dtype=torch.float32, device=dev)[:2]
+    inv = torch.empty(K, dtype=torch.float32, device=dev)
+    rr = (2 * r if p == NVFP4 else r)
+    lr_up = torch.empty((N, rr), dtype=torch.bfloat16, device=dev) if r else None
+    _check("svdq_pack_weight", load().svdq_pack_weight(
+        p, K, N, r, _ptr(W), _ptr(lam), _ptr(L1), _ptr(L2), float(act_tensor_scale), _ptr(codes),
+        _ptr(scales), _ptr(ts), _ptr(inv), _ptr(lr_up), _stream(stream)))
+    return PackedWeight(p, K, N, r, codes, scales, ts, inv, lr_up, float(act_tensor_scale))
+
+
+def quantize_act(x: torch.Tensor, pw: PackedWeight, L1: Optional[torch.Tensor], stream=None,
+                 out: Optional[QuantAct] = None) -> QuantAct:
+    """svdq_quantize_act: x bf16 [M, K] -> codes, scales, P."""
+    M, K = x.shape
+    p, r = pw.prec, pw.r
+    dev = x.device
+    if out is None:
+        out = QuantAct(p, M, K, r, torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                       torch.empty(max(scale_bytes(p, M, K), 16), dtype=torch.uint8, device=dev),
+                       torch.empty((M, r), dtype=torch.bfloat16, device=dev) if r else None)
+    _check("svdq_quantize_act", load().svdq_quantize_act(
+        p, M, K, r, _ptr(x), _ptr(pw.inv_lambda), float(pw.act_tensor_scale), _ptr(L1),
+        _ptr(out.codes), _ptr(out.scales), _ptr(out.P), _stream(stream)))
+    return out
+
+
+def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = None,
+                out_dtype: str = "bf16", stream=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """svdq_w4a4_linear: the 4-bit GEMM with the low-rank up-projection and bias fused."""
+    M, K, N = qa.M, qa.K, pw.N
+    if out is None:
+        if out_dtype == "bf16":
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.codes.device)
+        elif out_dtype == "f32":
+            out = torch.empty((M, N), dtype=torch.float32, device=qa.codes.device)
+        else:
+            out = torch.empty((M, N, K // 64), dtype=torch.int32, device=qa.codes.device)
+    _check("svdq_w4a4_linear", load().svdq_w4a4_linear(
+        pw.prec, M, K, N, pw.r, _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.P), _ptr(pw.codes),
+        _ptr(pw.scales), _ptr(pw.tensor_scale), _ptr(pw.lr_up), _ptr(bias), _ptr(out),
+        _OUT[out_dtype], _stream(stream)))
+    return out
+
+
+def svdq_linear(x: torch.Tensor, pw: PackedWeight, L1: Optional[torch.Tensor],
+                bias: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The whole layer: quantize_act then w4a4_linear (two launches)."""
+    return w4a4_linear(quantize_act(x, pw, L1, stream), pw, bias, stream=stream)
+
+
+@dataclass
+class AwqWeight:
+    K: int
+    N: int
+    q: torch.Tensor       # uint8 [N, K/2]
+    scales: torch.Tensor  # bf16 [N, K/64]
+    zeros: torch.Tensor   # bf16 [N, K/64]
+
+
+def awq_pack_weight(W: torch.Tensor, stream=None) -> AwqWeight:
+    K, N = W.shape
+    dev = W.device
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    s = torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev)
+    z = torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev)
+    _check("awq_pack_weight", load().awq_pack_weight(K, N, _ptr(W), _ptr(q), _ptr(s), _ptr(z),
+                                                     _stream(stream)))
+    return AwqWeight(K, N, q, s, z)
+
+
+def awq_w4a16_linear(x: torch.Tensor, w: AwqWeight, bias: Optional[torch.Tensor] = None, stream=None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    _check("awq_w4a16_linear", load().awq_w4a16_linear(
+        M, K, w.N, _ptr(x), _ptr(w.q), _ptr(w.scales), _ptr(w.zeros), _ptr(bias), _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def device_error() -> int:
+    """Reads and clears the device error word; raises SvdqError if it was set."""
+    bits = C.c_uint(0)
+    st = load().svdq_device_error(C.byref(bits))
+    if st not in (0, int(Status.TIMEOUT), int(Status.CUDA)):
+        _check("svdq_device_error", st)
+    if st:
+        raise SvdqError("svdq_device_error", st, f"device error word = {bits.value:#x}")
+    return bits.value
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load().svdq_set_wait_limit_ns(int(ns))
+
+
+def probe_convert(x: torch.Tensor, e2m1: bool = True, e4m3: bool = True, bf16: bool = True, stream=None):
+    n = x.numel()
+    o1 = torch.empty(n, dtype=torch.uint8, device=x.device) if e2m1 else None
+    o2 = torch.empty(n, dtype=torch.uint8, device=x.device) if e4m3 else None
+    o3 = torch.empty(n, dtype=torch.int16, device=x.device) if bf16 else None
+    _check("svdq_probe_convert", load().svdq_probe_convert(_ptr(x), n, _ptr(o1), _ptr(o2), _ptr(o3),
+                                                           _stream(stream)))
+    return o1, o2, o3
+
+
+def probe_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check("svdq_probe_wait_timeout", load().svdq_probe_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def debug_force_arch(major: int, minor: int = 0) -> None:
+    load().svdq_debug_force_arch(int(major), int(minor))

@@ -1,0 +1,87 @@
+// Launch interfaces of the library's kernels (host side of csrc/*.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace svdq {
+
+struct QuantActArgs {
+  const uint16_t* x;          // bf16 [M, K]
+  const float* inv_lambda;    // [K]
+  const uint16_t* L1;         // bf16 [K, r]
+  uint8_t* codes;             // [M, K/2]
+  void* scales;               // NVFP4 tiled e4m3 / INT4 bf16 [M, K/64]
+  uint16_t* P;                // bf16 [M, r]
+  int M, K, r;
+  float s_tx;
+};
+cudaError_t launch_quant_act(int prec, const QuantActArgs& a, cudaStream_t s);
+
+struct PackArgs {
+  const float* W;             // [K, N]
+  const float* lambda;        // [K]
+  const uint16_t* L1;         // [K, r]
+  const uint16_t* L2;         // [r, N]
+  uint8_t* codes;             // [N, K/2]
+  void* scales;
+  float* tensor_scale;        // [2]
+  float* inv_lambda;          // [K]
+  uint16_t* lr_up;            // [N, rr]
+  int K, N, r;
+  float s_tx;
+};
+cudaError_t launch_pack(int prec, const PackArgs& a, size_t scale_bytes, cudaStream_t s);
+
+struct AwqPackArgs {
+  const float* W;
+  uint8_t* q;
+  uint16_t* s;
+  uint16_t* z;
+  int K, N;
+};
+cudaError_t launch_awq_pack(const AwqPackArgs& a, cudaStream_t s);
+
+struct AwqArgs {
+  const uint16_t* x;
+  const uint8_t* q;
+  const uint16_t* s;
+  const uint16_t* z;
+  const uint16_t* bias;
+  uint16_t* y;
+  int M, K, N;
+};
+cudaError_t launch_awq(const AwqArgs& a, cudaStream_t s);
+
+struct GemmArgs {
+  const uint8_t* x_codes;
+  const void* x_scales;
+  const uint16_t* P;
+  const uint8_t* w_codes;
+  const void* w_scales;
+  const float* tensor_scale;  // [2] = {s_tw, s_tx}
+  const uint16_t* lr_up;
+  const uint16_t* bias;
+  void* y;
+  int M, K, N, r;
+  int out;                    // svdq_out_dtype
+  unsigned* err;
+  unsigned long long wait_ns;
+  int num_sms;
+};
+cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_gemm_int4(const GemmArgs& a, cudaStream_t s);
+
+cudaError_t launch_probe_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3,
+                                 uint16_t* bf16, cudaStream_t s);
+cudaError_t launch_probe_wait(unsigned* err, unsigned long long limit_ns, cudaStream_t s);
+
+// Host helper: encode a 2-D tiled tensor map (driver entry point looked up at
+// run time; no link-time dependency on libcuda).
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swz);
+
+}  // namespace svdq

@@ -9,6 +9,7 @@ checkpoint (smoothing vector and rank-r factors, see ``inputs``).
 
 from .inputs import (  # noqa: F401
     CONFIGS,
+    config_layer,
     awq_inputs,
     bf16_bits,
     bf16_bits_to_f32,

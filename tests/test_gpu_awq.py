@@ -1,0 +1,74 @@
+"""GPU parity of the awq_w4a16 path (pack bit-exact, output within the float
+tolerance rule) against the CPU oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import bit_w4a4_quantized_nvfp4_b200 as svdq
+from tests._util import check_bf16_output
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_w4a4_quantized_nvfp4_b200 import build
+
+    build.build()
+    svdq.load()
+
+
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bf16_np(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.fixture(scope="module")
+def full_weight():
+    c = synth.CONFIGS["c2_awq_gemv"]
+    d = synth.awq_inputs(c["seed"], 16, c["K"], c["N"])
+    pk = oracle.awq_pack_weight(d["W"])
+    w = svdq.awq_pack_weight(torch.from_numpy(d["W"]).cuda())
+    torch.cuda.synchronize()
+    return d, pk, w
+
+
+def test_awq_pack_full_size_bit_exact(full_weight):
+    d, pk, w = full_weight
+    assert np.array_equal(w.q.cpu().numpy(), pk["q"])
+    assert np.array_equal(bf16_np(w.scales), pk["s"])
+    assert np.array_equal(bf16_np(w.zeros), pk["z"])
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 16])
+def test_awq_gemv_full_size(full_weight, M):
+    d, pk, w = full_weight
+    x = d["x"][:M]
+    y = svdq.awq_w4a16_linear(bf16_dev(x), w)
+    torch.cuda.synchronize()
+    yo = oracle.awq_linear(x, pk)
+    check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
+
+
+@pytest.mark.parametrize("M,K,N", [(3, 128, 72), (17, 192, 136), (40, 64, 8), (1, 4096, 24)])
+def test_awq_ragged_shapes_with_bias(M, K, N):
+    d = synth.awq_inputs(31, M, K, N)
+    b = synth.bf16_bits(np.linspace(-0.05, 0.05, N))
+    pk = oracle.awq_pack_weight(d["W"])
+    w = svdq.awq_pack_weight(torch.from_numpy(d["W"]).cuda())
+    big = torch.full((M * N + 1024,), 777.0, dtype=torch.bfloat16, device="cuda")
+    y = big[: M * N].view(M, N)
+    svdq.awq_w4a16_linear(bf16_dev(d["x"]), w, bf16_dev(b), out=y)
+    torch.cuda.synchronize()
+    assert (big[M * N:] == 777.0).all()
+    assert np.array_equal(w.q.cpu().numpy(), pk["q"])
+    yo = oracle.awq_linear(d["x"], pk, b)
+    check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))

@@ -68,17 +68,24 @@ using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, voi
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
-                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+namespace {
+EncodeFn encode_fn() {
   static EncodeFn fn = nullptr;
   if (!fn) {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !f)
-      return false;
-    fn = reinterpret_cast<EncodeFn>(f);
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && f)
+      fn = reinterpret_cast<EncodeFn>(f);
   }
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
@@ -86,6 +93,20 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
   std::memset(map, 0, sizeof(*map));
   return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1, stride2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  std::memset(map, 0, sizeof(*map));
+  return fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace svdq
@@ -154,7 +175,8 @@ svdq_status svdq_quantize_act(svdq_precision p, int M, int K, int r, const uint1
   if (!aligned16(x) || !aligned16(inv_lambda) || !aligned16(x_codes) || !aligned16(x_scales) ||
       (r > 0 && (!aligned16(L1) || !aligned16(P))))
     return SVDQ_ERR_ALIGN;
-  if ((st = device_info(nullptr, nullptr)) != SVDQ_OK) return st;
+  unsigned* err = nullptr;
+  if ((st = device_info(&err, nullptr)) != SVDQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (p == SVDQ_NVFP4 && M % 128) {
     // zero the scales of the padding rows of the last 128-row block
@@ -163,7 +185,7 @@ svdq_status svdq_quantize_act(svdq_precision p, int M, int K, int r, const uint1
       return SVDQ_ERR_CUDA;
   }
   QuantActArgs a{x, inv_lambda, L1, x_codes, x_scales, P, M, K, r, act_tensor_scale};
-  return from_cuda(launch_quant_act((int)p, a, s));
+  return from_cuda(launch_quant_act((int)p, a, err, g_wait_ns.load(), s));
 }
 
 svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const uint8_t* x_codes,

@@ -18,7 +18,8 @@ struct QuantActArgs {
   int M, K, r;
   float s_tx;
 };
-cudaError_t launch_quant_act(int prec, const QuantActArgs& a, cudaStream_t s);
+cudaError_t launch_quant_act(int prec, const QuantActArgs& a, unsigned* err, unsigned long long wait_ns,
+                             cudaStream_t s);
 
 struct PackArgs {
   const float* W;             // [K, N]
@@ -83,5 +84,9 @@ cudaError_t launch_probe_wait(unsigned* err, unsigned long long limit_ns, cudaSt
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                   CUtensorMapSwizzle swz);
+// 3-D tiled tensor map without swizzle: dims {d0, d1, d2}, byte strides of
+// dims 1 and 2, box {b0, b1, b2}.
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                  uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2);
 
 }  // namespace svdq

@@ -1,6 +1,6 @@
 // K1 — the fused activation pass of the SVDQuant W4A4 layer.
 //
-// One coalesced, vectorised pass over x computes, for every row:
+// One coalesced pass over x computes, for every row:
 //   x_hat = bf16(x * inv_lambda)                       (smoothing)
 //   4-bit codes and group scales of x_hat              (NVFP4 g16 / INT4 g64)
 //   P = bf16(x_hat L1)                                  (low-rank down-projection)
@@ -8,22 +8,25 @@
 // (blog "Introducing Nunchaku 4-bit inference in Diffusers", section
 // "Background: SVDQuant and Nunchaku", figure caption).
 //
-// Work split: a CTA owns 32 rows and walks K in chunks of 256 columns. Each of
-// its 8 warps quantises 4 rows; lane l handles 8 consecutive columns of a row
-// (one 16-byte load), so a warp reads a 512-byte row segment per load and
-// writes 128 contiguous bytes of codes. x_hat is staged in shared memory and
-// multiplied by the L1 chunk on tensor cores (mma.sync bf16, fp32 accumulate);
-// the 8 warps split the chunk 2 (row tiles) x 4 (K quarters) and the K
-// quarters are summed in a fixed order at the end.
+// Work split: a CTA owns 32 rows and walks K in chunks of 256 columns through
+// a multi-stage TMA pipeline (each stage: the 32 x 256 x tile and the matching
+// 256 x r L1 tile, the latter with the TMA swizzle that makes the ldmatrix
+// reads below bank-conflict free), so that several chunks are in flight per SM.
+// Each of the 8 warps quantises 4 rows; lane l handles 8 consecutive columns of
+// a row, so a warp writes 128 contiguous bytes of codes per row. x_hat is
+// staged in shared memory and multiplied by the L1 tile on tensor cores
+// (mma.sync bf16, fp32 accumulate); the warps split each chunk 2 (row tiles) x
+// 4 (K quarters) and the K quarters are summed in a fixed order at the end.
 #include "device.cuh"
 #include "kernels.h"
 
 namespace svdq {
 namespace {
 
-constexpr int kRows = 32;     // rows per CTA
-constexpr int kChunk = 256;   // K columns per step
-constexpr int kXhStride = kChunk + 8;  // bf16 elements per staged row (bank spread)
+constexpr int kRows = 32;              // rows per CTA
+constexpr int kChunk = 256;            // K columns per stage
+constexpr int kXhStride = kChunk + 8;  // bf16 elements per staged x_hat row (bank spread)
+constexpr int kXBytes = kRows * kChunk * 2;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -42,23 +45,38 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
+// two fp32 -> bf16x2 (round to nearest even); `lo` in bits 0..15
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
+
+template <int NT>
+struct StageLayout {
+  static constexpr int kR = NT * 8;
+  static constexpr int kL1Bytes = NT ? kChunk * kR * 2 : 0;
+  static constexpr int kStageBytes = ((kXBytes + kL1Bytes + 1023) / 1024) * 1024;
+  static constexpr int kStages = (kR <= 32) ? 4 : 3;
+  // L1 tile rows are 2r bytes; the TMA swizzle span equals the row (32/64/128 B)
+  static constexpr uint32_t kSwzMask = kR <= 16 ? 1u : (kR == 32 ? 3u : 7u);
+};
 
 // PREC 0 = NVFP4 (group 16, E4M3 scales in the tiled layout), 1 = INT4
 // (group 64, bf16 scales row-major). NT = r / 8 tiles of the P output.
 template <int PREC, int NT>
-__global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(smem);                 // [32][264]
-  constexpr int kR = NT * 8;
-  constexpr int kL1Stride = kR + 8;
-  __nv_bfloat16* l1s = xh + kRows * kXhStride;                                // [256][r+8]
-  float* red = reinterpret_cast<float*>(l1s + (NT ? kChunk * kL1Stride : 0));  // [4][32][r]
+__global__ void __launch_bounds__(256, 1)
+quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
+                 QuantActArgs a, unsigned* err, unsigned long long wait_ns) {
+  using L = StageLayout<NT>;
+  constexpr int kR = L::kR;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* stages = base;                                                      // S x kStageBytes
+  __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(base + S * L::kStageBytes);  // [32][264]
+  float* red = reinterpret_cast<float*>(xh + kRows * kXhStride);               // [4][32][r]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + (NT ? 4 * kRows * kR : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * kRows;
@@ -66,48 +84,40 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
   const int nchunks = (K + kChunk - 1) / kChunk;
   const float s_tx = a.s_tx;
   const float six_t = __fmul_rn(6.0f, s_tx);
+  const uint32_t stage_tx = kXBytes + L::kL1Bytes;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_x);
+    if (NT) tma_prefetch_desc(&tm_l1);
+    for (int c = 0; c < S && c < nchunks; ++c) {
+      uint8_t* st = stages + c * L::kStageBytes;
+      mbar_expect_tx(&full[c], stage_tx);
+      tma_load_2d(st, &tm_x, &full[c], c * kChunk, row0);
+      if (NT) tma_load_2d(st + kXBytes, &tm_l1, &full[c], 0, c * kChunk);
+    }
+  }
+  __syncthreads();
 
   float acc[NT > 0 ? NT : 1][4];
 #pragma unroll
   for (int t = 0; t < (NT > 0 ? NT : 1); ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
-  // prefetch chunk 0
-  uint4 xv[4];
-  auto load_chunk = [&](int c, uint4 (&v)[4]) {
-    const int col = c * kChunk + lane * 8;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = row0 + warp + 8 * i;
-      if (m < M && col < K)
-        v[i] = ldg_stream(a.x + (size_t)m * K + col);
-      else
-        v[i] = make_uint4(0, 0, 0, 0);
-    }
-  };
-  load_chunk(0, xv);
-
+  bool ok = true;
   for (int c = 0; c < nchunks; ++c) {
+    const int s = c % S;
+    uint8_t* st = stages + s * L::kStageBytes;
+    if (!mbar_wait(&full[s], (c / S) & 1, wait_ns, err)) ok = false;
+    // every thread reaches the barriers below whatever happened, so that no
+    // thread waits on one that others skipped
     const int col = c * kChunk + lane * 8;
-    const bool col_ok = col < K;
-    uint4 cur[4] = {xv[0], xv[1], xv[2], xv[3]};
-    if (c + 1 < nchunks) load_chunk(c + 1, xv);
-
-    // stage the L1 chunk [256 x r] (rows beyond K are zero)
-    if constexpr (NT > 0) {
-      constexpr int kVecPerRow = kR / 8;  // 16-byte vectors per L1 row
-      for (int v = threadIdx.x; v < kChunk * kVecPerRow; v += blockDim.x) {
-        const int kr = v / kVecPerRow, cv = v % kVecPerRow;
-        const int kg = c * kChunk + kr;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (kg < K) val = *reinterpret_cast<const uint4*>(a.L1 + (size_t)kg * kR + cv * 8);
-        *reinterpret_cast<uint4*>(l1s + kr * kL1Stride + cv * 8) = val;
-      }
-    }
+    const bool col_ok = ok && col < K;
 
     float il[8];
     if (col_ok) {
-      const float4 i0 = *reinterpret_cast<const float4*>(a.inv_lambda + col);
-      const float4 i1 = *reinterpret_cast<const float4*>(a.inv_lambda + col + 4);
+      const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + col));
+      const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + col + 4));
       il[0] = i0.x; il[1] = i0.y; il[2] = i0.z; il[3] = i0.w;
       il[4] = i1.x; il[5] = i1.y; il[6] = i1.z; il[7] = i1.w;
     } else {
@@ -119,20 +129,20 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
     for (int i = 0; i < 4; ++i) {
       const int lr = warp + 8 * i;  // local row
       const int m = row0 + lr;
-      const uint32_t w[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+      const uint4 xv = *reinterpret_cast<const uint4*>(st + lr * (kChunk * 2) + lane * 16);
+      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
       float xf[8];
       uint32_t hb[4];
-      float amax = 0.f;
+      __nv_bfloat162 amax2 = __float2bfloat162_rn(0.f);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float x0 = bf16_bits_to_f32(w[j] & 0xFFFFu), x1 = bf16_bits_to_f32(w[j] >> 16);
-        const uint32_t h0 = f32_to_bf16_bits(__fmul_rn(x0, il[2 * j]));
-        const uint32_t h1 = f32_to_bf16_bits(__fmul_rn(x1, il[2 * j + 1]));
-        hb[j] = h0 | (h1 << 16);
-        xf[2 * j] = bf16_bits_to_f32(h0);
-        xf[2 * j + 1] = bf16_bits_to_f32(h1);
-        amax = fmaxf(amax, fmaxf(fabsf(xf[2 * j]), fabsf(xf[2 * j + 1])));
+        const float x0 = __uint_as_float(w[j] << 16), x1 = __uint_as_float(w[j] & 0xFFFF0000u);
+        hb[j] = pack_bf16x2(__fmul_rn(x0, il[2 * j]), __fmul_rn(x1, il[2 * j + 1]));
+        xf[2 * j] = __uint_as_float(hb[j] << 16);
+        xf[2 * j + 1] = __uint_as_float(hb[j] & 0xFFFF0000u);
+        amax2 = __hmax2(amax2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&hb[j])));
       }
+      float amax = fmaxf(__low2float(amax2), __high2float(amax2));
       *reinterpret_cast<uint4*>(xh + lr * kXhStride + lane * 8) = make_uint4(hb[0], hb[1], hb[2], hb[3]);
 
       if (PREC == 0) {
@@ -154,7 +164,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
         if (m < M && col_ok) {
           *reinterpret_cast<uint32_t*>(a.codes + (size_t)m * (K / 2) + col / 2) = code;
           if ((lane & 7) == 0) {
-            const int ka = (c * kChunk + lane * 8) / 64;  // atom index along K
+            const int ka = col / 64;  // atom index along K
             const size_t atom = ((size_t)(m / 128) * (K / 64) + ka) * 512;
             const uint32_t word = sf | (s1 << 8) | (s2 << 16) | (s3 << 24);
             *reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(a.scales) + atom + 16 * (m % 32) +
@@ -189,23 +199,31 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
     if constexpr (NT > 0) {
       // tensor-core partial products: warp -> (row tile, K quarter)
       const int mt = warp & 1, kq = warp >> 1;
+      const uint32_t l1base = smem_u32(st + kXBytes);
 #pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const int k0 = (kq * 4 + s) * 16;
+      for (int ks = 0; ks < 4; ++ks) {
+        const int k0 = (kq * 4 + ks) * 16;
         uint32_t a0, a1, a2, a3;
         const int ar = mt * 16 + (lane & 15), ac = k0 + (lane >> 4) * 8;
         ldsm_x4(smem_u32(xh + ar * kXhStride + ac), a0, a1, a2, a3);
 #pragma unroll
         for (int t = 0; t < NT; t += 2) {
           uint32_t b0, b1, b2, b3;
-          const int br = k0 + (lane & 7) + ((lane >> 3) & 1) * 8, bc = t * 8 + (lane >> 4) * 8;
-          ldsm_x4_t(smem_u32(l1s + br * kL1Stride + bc), b0, b1, b2, b3);
+          const int br = k0 + (lane & 7) + ((lane >> 3) & 1) * 8, bc = t + (lane >> 4);  // bc in 16-byte chunks
+          const uint32_t off = (uint32_t)(br * (2 * kR) + 16 * bc);
+          ldsm_x4_t(l1base + (off ^ (((off >> 7) & L::kSwzMask) << 4)), b0, b1, b2, b3);
           mma_16816(acc[t], a0, a1, a2, a3, b0, b1);
           mma_16816(acc[t + 1], a0, a1, a2, a3, b2, b3);
         }
       }
     }
     __syncthreads();
+    // stage s is free: refill it with chunk c + S
+    if (threadIdx.x == 0 && ok && c + S < nchunks) {
+      mbar_expect_tx(&full[s], stage_tx);
+      tma_load_2d(st, &tm_x, &full[s], (c + S) * kChunk, row0);
+      if (NT) tma_load_2d(st + kXBytes, &tm_l1, &full[s], 0, (c + S) * kChunk);
+    }
   }
 
   if constexpr (NT > 0) {
@@ -215,17 +233,17 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       const int j = t * 8 + 2 * t4;
-      float* base = red + (size_t)kq * kRows * kR;
-      base[(mt * 16 + g) * kR + j] = acc[t][0];
-      base[(mt * 16 + g) * kR + j + 1] = acc[t][1];
-      base[(mt * 16 + g + 8) * kR + j] = acc[t][2];
-      base[(mt * 16 + g + 8) * kR + j + 1] = acc[t][3];
+      float* rb = red + (size_t)kq * kRows * kR;
+      rb[(mt * 16 + g) * kR + j] = acc[t][0];
+      rb[(mt * 16 + g) * kR + j + 1] = acc[t][1];
+      rb[(mt * 16 + g + 8) * kR + j] = acc[t][2];
+      rb[(mt * 16 + g + 8) * kR + j + 1] = acc[t][3];
     }
     __syncthreads();
     for (int e = threadIdx.x; e < kRows * kR; e += blockDim.x) {
       const int lr = e / kR, j = e % kR;
       const int m = row0 + lr;
-      if (m >= M) continue;
+      if (m >= M || !ok) continue;
       float v = red[e];
       v += red[kRows * kR + e];
       v += red[2 * kRows * kR + e];
@@ -236,35 +254,49 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantActArgs a) {
 }
 
 template <int PREC, int NT>
-cudaError_t launch_t(const QuantActArgs& a, cudaStream_t s) {
-  constexpr int kR = NT * 8;
-  const size_t smem = (size_t)kRows * kXhStride * 2 + (NT ? (size_t)kChunk * (kR + 8) * 2 : 0) +
-                      (size_t)4 * kRows * kR * 4;
+cudaError_t launch_t(const QuantActArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s) {
+  using L = StageLayout<NT>;
+  constexpr int kR = L::kR;
+  CUtensorMap tm_x, tm_l1;
+  if (!make_tmap_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, a.K, a.M, (uint64_t)a.K * 2, kChunk, kRows,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (NT) {
+    const CUtensorMapSwizzle swz = kR == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                            : (kR == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!make_tmap_2d(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L1, kR, a.K, (uint64_t)kR * 2, kR, kChunk, swz))
+      return cudaErrorInvalidValue;
+  } else {
+    tm_l1 = tm_x;
+  }
+  const size_t smem = 1024 + (size_t)L::kStages * L::kStageBytes + (size_t)kRows * kXhStride * 2 +
+                      (NT ? (size_t)4 * kRows * kR * 4 : 0) + 64;
   auto k = quant_act_kernel<PREC, NT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = (a.M + kRows - 1) / kRows;
-  k<<<grid, 256, smem, s>>>(a);
+  k<<<grid, 256, smem, s>>>(tm_x, tm_l1, a, err, wait_ns);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_quant_act(int prec, const QuantActArgs& a, cudaStream_t s) {
+cudaError_t launch_quant_act(int prec, const QuantActArgs& a, unsigned* err, unsigned long long wait_ns,
+                             cudaStream_t s) {
   const int nt = a.r / 8;
   if (prec == 0) {
     switch (nt) {
-      case 0: return launch_t<0, 0>(a, s);
-      case 2: return launch_t<0, 2>(a, s);
-      case 4: return launch_t<0, 4>(a, s);
+      case 0: return launch_t<0, 0>(a, err, wait_ns, s);
+      case 2: return launch_t<0, 2>(a, err, wait_ns, s);
+      case 4: return launch_t<0, 4>(a, err, wait_ns, s);
     }
   } else {
     switch (nt) {
-      case 0: return launch_t<1, 0>(a, s);
-      case 2: return launch_t<1, 2>(a, s);
-      case 4: return launch_t<1, 4>(a, s);
-      case 6: return launch_t<1, 6>(a, s);
-      case 8: return launch_t<1, 8>(a, s);
+      case 0: return launch_t<1, 0>(a, err, wait_ns, s);
+      case 2: return launch_t<1, 2>(a, err, wait_ns, s);
+      case 4: return launch_t<1, 4>(a, err, wait_ns, s);
+      case 6: return launch_t<1, 6>(a, err, wait_ns, s);
+      case 8: return launch_t<1, 8>(a, err, wait_ns, s);
     }
   }
   return cudaErrorInvalidValue;

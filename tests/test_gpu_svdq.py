@@ -223,3 +223,37 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert svdq.device_error() == 0  # cleared
     # the context is still usable
     test_nvfp4_layer_matches_oracle(*CASES[4])
+
+
+# ------------------------------------------------------------------ INT4 GEMM
+@pytest.mark.parametrize("M,K,N,r", [(256, 1024, 512, 32), (37, 192, 72, 16), (130, 256, 264, 64), (3, 64, 8, 0)])
+def test_int4_linear_matches_oracle(M, K, N, r):
+    d = synth.svdq_layer(26, M, K, N, r, x_out_frac=0.02, x_out_scale=30.0)
+    pw, qa, y = run_layer("int4", d)
+    w, a, yo = oracle_layer("int4", d)
+    compare_pack_and_act("int4", d, pw, qa, w, a)
+    check_bf16_output(as_f32(bf16_np(y)), yo, as_f32(oracle.bf16_rn(yo)))
+    _, _, y32 = run_layer("int4", d, out_dtype="f32")
+    check_f32_output(y32.cpu().numpy(), yo)
+    # the int32 group dot products are exact
+    gs = svdq.w4a4_linear(qa, pw, None, out_dtype="i32_groups")
+    torch.cuda.synchronize()
+    assert np.array_equal(gs.cpu().numpy(), oracle.int4_group_sums(a["codes"], w["codes"]))
+
+
+def test_c5_int4_full_size():
+    """INT4 workload (M4608 K3072 N9216 r32, g64): codes and scales in full, y
+    on 128 seeded rows, exact int32 group sums on the first 48 rows."""
+    c = synth.CONFIGS["c5_qkv_int4"]
+    d = synth.config_layer("c5_qkv_int4")
+    pw, qa, y = run_layer("int4", d)
+    rows = np.sort(np.random.default_rng(5).choice(c["M"], 128, replace=False)).astype(np.int32)
+    w, a, yo = oracle_layer("int4", d, rows=rows)
+    compare_pack_and_act("int4", d, pw, qa, w, a)
+    check_bf16_output(as_f32(bf16_np(y))[rows], yo, as_f32(oracle.bf16_rn(yo)))
+    sub = svdq.QuantAct(qa.prec, 48, qa.K, qa.r, qa.codes[:48].contiguous(),
+                        qa.scales[: 48 * (qa.K // 64) * 2].contiguous(),
+                        qa.P[:48].contiguous() if qa.P is not None else None)
+    gs = svdq.w4a4_linear(sub, pw, None, out_dtype="i32_groups")
+    torch.cuda.synchronize()
+    assert np.array_equal(gs.cpu().numpy(), oracle.int4_group_sums(a["codes"][:48], w["codes"]))

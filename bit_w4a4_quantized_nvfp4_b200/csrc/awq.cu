@@ -87,27 +87,31 @@ __global__ void __launch_bounds__(128) awq_kernel(AwqArgs a) {
         }
       }
 
-      // stage activations of this chunk in fragment order
+      // stage activations of this chunk in fragment order: one 16-byte load
+      // holds x[m, 64g + 16t + 8h .. +7], i.e. the pairs (e, e+4) of steps
+      // 2h (e = 8h, 8h+1) and 2h+1 (e = 8h+2, 8h+3)
       __syncthreads();
-      const int words = mt_count * kChunkGroups * 4 * 4 * 8 * 2;
-      for (int wi = threadIdx.x; wi < words; wi += blockDim.x) {
-        int r = wi;
-        const int half = r & 1; r >>= 1;
-        const int mm = r & 7; r >>= 3;
+      const int loads = mt_count * 8 * kChunkGroups * 8;  // (m, group, t, h)
+      for (int li = threadIdx.x; li < loads; li += blockDim.x) {
+        int r = li;
+        const int h = r & 1; r >>= 1;
         const int tt = r & 3; r >>= 2;
-        const int st = r & 3; r >>= 2;
-        const int gg = r % kChunkGroups;
-        const int mt = r / kChunkGroups;
+        const int gg = r % kChunkGroups; r /= kChunkGroups;
+        const int mm = r & 7;
+        const int mt = r >> 3;
         const int m = m0 + mt * 8 + mm;
-        const int g = g0 + gg;
-        // slot pairs of step st: (e, e+4) with e = {0,1 | 2,3 | 8,9 | 10,11}[2 st + half]
-        const int e = (st >> 1) * 8 + (st & 1) * 2 + half;
-        uint32_t v = 0;
-        if (m < M && gg < gcount) {
-          const uint16_t* xr = a.x + (size_t)m * K + g * 64 + tt * 16;
-          v = (uint32_t)xr[e] | ((uint32_t)xr[e + 4] << 16);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (m < M && gg < gcount)
+          v = *reinterpret_cast<const uint4*>(a.x + (size_t)m * K + (g0 + gg) * 64 + tt * 16 + h * 8);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        // element e' (0..7) of the load: bf16 halves of w[e'/2]
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {          // pair (q, q+4) of the load
+          const uint32_t lo = (q & 1) ? (w[q >> 1] >> 16) : (w[q >> 1] & 0xFFFFu);
+          const uint32_t hi = (q & 1) ? (w[2 + (q >> 1)] >> 16) : (w[2 + (q >> 1)] & 0xFFFFu);
+          const int st = 2 * h + (q >> 1), half = q & 1;
+          xs[((((mt * kChunkGroups + gg) * 4 + st) * 4 + tt) * 8 + mm) * 2 + half] = lo | (hi << 16);
         }
-        xs[wi] = v;
       }
       __syncthreads();
 

@@ -76,6 +76,11 @@ struct Params {
   unsigned long long wait_ns;
 };
 
+// Bounded wait by a whole warp with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long ns, unsigned* err) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ns, err));
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -167,20 +172,24 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
-    if (leader && lane == 0) {
+    // The whole warp walks the loop; one lane issues the tcgen05 ops.
+    if (leader) {
       uint32_t it = 0;
       bool ok = true;
       int i = 0;
       for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++i) {
         const uint32_t acc = tmem + ((i & 1) ? kAccCol1 : kAccCol0);
-        if (i > 0 && !mbar_wait_cluster(&sm.acc_free, (i - 1) & 1, p.wait_ns, p.err)) { ok = false; break; }
+        if (i > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(&sm.acc_free, (i - 1) & 1, p.wait_ns, p.err))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
-          tc_fence_after();
+          if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
           const uint32_t st = smem_u32(sm.stage[s]);
           const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfaBytes;
+          if (lane == 0) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             tc_cp_32x128b_warpx4_pair(tmem + kSfaCol + 4 * j, make_sdesc(sfa + 512 * j, 512, 128, kLayoutNone));
@@ -196,28 +205,34 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                            (kb > 0 || j > 0) ? 1u : 0u);
           }
           tc_commit_pair(&sm.empty[s], 0x3);
+          }
+          __syncwarp();
         }
         if (!ok) break;
         if (has_lr) {
           const int s = it % kStages;
-          if (!mbar_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
-          tc_fence_after();
+          if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
           const uint32_t st = smem_u32(sm.stage[s]);
           const int half = p.r / 16;  // k16 steps per copy of P
-          for (int k = 0; k < 2 * half; ++k) {
-            const int kp = k % half;
-            const uint64_t ad = make_sdesc(st + 2 * kp * BM * 16, BM * 16, 128, kLayoutNone);
-            const uint64_t bd = make_sdesc(st + kABytes + 2 * k * BM * 16, BM * 16, 128, kLayoutNone);
-            mma_bf16_pair(acc, ad, bd, kIdescBf16, 1u);
+          if (lane == 0) {
+            for (int k = 0; k < 2 * half; ++k) {
+              const int kp = k % half;
+              const uint64_t ad = make_sdesc(st + 2 * kp * BM * 16, BM * 16, 128, kLayoutNone);
+              const uint64_t bd = make_sdesc(st + kABytes + 2 * k * BM * 16, BM * 16, 128, kLayoutNone);
+              mma_bf16_pair(acc, ad, bd, kIdescBf16, 1u);
+            }
+            tc_commit_pair(&sm.empty[s], 0x3);
           }
-          tc_commit_pair(&sm.empty[s], 0x3);
+          __syncwarp();
           ++it;
         }
-        tc_commit_pair(&sm.acc_full[i & 1], 0x3);
+        if (lane == 0) tc_commit_pair(&sm.acc_full[i & 1], 0x3);
+        __syncwarp();
       }
       // every MMA issued has completed before tensor memory is freed
-      tc_commit_pair(&sm.mma_done, 0x1);
-      (void)mbar_wait(&sm.mma_done, 0, p.wait_ns, p.err);
+      if (lane == 0) tc_commit_pair(&sm.mma_done, 0x1);
+      __syncwarp();
+      (void)warp_wait(&sm.mma_done, 0, p.wait_ns, p.err);
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)

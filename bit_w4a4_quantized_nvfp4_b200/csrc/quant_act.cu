@@ -12,11 +12,11 @@
 // a multi-stage TMA pipeline (each stage: the 32 x 256 x tile and the matching
 // 256 x r L1 tile, the latter with the TMA swizzle that makes the ldmatrix
 // reads below bank-conflict free), so that several chunks are in flight per SM.
-// Each of the 8 warps quantises 4 rows; lane l handles 8 consecutive columns of
-// a row, so a warp writes 128 contiguous bytes of codes per row. x_hat is
+// Each of the 16 warps quantises 2 rows; lane l handles 8 consecutive columns
+// of a row, so a warp writes 128 contiguous bytes of codes per row. x_hat is
 // staged in shared memory and multiplied by the L1 tile on tensor cores
 // (mma.sync bf16, fp32 accumulate); the warps split each chunk 2 (row tiles) x
-// 4 (K quarters) and the K quarters are summed in a fixed order at the end.
+// 8 (K eighths) and the eighths are summed in a fixed order at the end.
 #include "device.cuh"
 #include "kernels.h"
 
@@ -27,6 +27,10 @@ constexpr int kRows = 32;              // rows per CTA
 constexpr int kChunk = 256;            // K columns per stage
 constexpr int kXhStride = kChunk + 8;  // bf16 elements per staged x_hat row (bank spread)
 constexpr int kXBytes = kRows * kChunk * 2;
+constexpr int kThreadsQA = 512;
+constexpr int kWarpsQA = kThreadsQA / 32;
+constexpr int kRowsPerWarp = kRows / kWarpsQA;    // 2
+constexpr int kKParts = kWarpsQA / 2;             // K splits of a chunk for the P product
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -65,7 +69,7 @@ struct StageLayout {
 // PREC 0 = NVFP4 (group 16, E4M3 scales in the tiled layout), 1 = INT4
 // (group 64, bf16 scales row-major). NT = r / 8 tiles of the P output.
 template <int PREC, int NT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kThreadsQA, 1)
 quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
                  QuantActArgs a, unsigned* err, unsigned long long wait_ns) {
   using L = StageLayout<NT>;
@@ -75,8 +79,8 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = base;                                                      // S x kStageBytes
   __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(base + S * L::kStageBytes);  // [32][264]
-  float* red = reinterpret_cast<float*>(xh + kRows * kXhStride);               // [4][32][r]
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + (NT ? 4 * kRows * kR : 0));
+  float* red = reinterpret_cast<float*>(xh + kRows * kXhStride);               // [kKParts][32][r]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + (NT ? kKParts * kRows * kR : 0));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * kRows;
@@ -126,8 +130,8 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
 
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int lr = warp + 8 * i;  // local row
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+      const int lr = warp + kWarpsQA * i;  // local row
       const int m = row0 + lr;
       const uint4 xv = *reinterpret_cast<const uint4*>(st + lr * (kChunk * 2) + lane * 16);
       const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -197,12 +201,13 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     __syncthreads();
 
     if constexpr (NT > 0) {
-      // tensor-core partial products: warp -> (row tile, K quarter)
+      // tensor-core partial products: warp -> (row tile, K eighth)
       const int mt = warp & 1, kq = warp >> 1;
       const uint32_t l1base = smem_u32(st + kXBytes);
+      constexpr int kSteps = kChunk / 16 / kKParts;  // k16 steps per warp and chunk
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const int k0 = (kq * 4 + ks) * 16;
+      for (int ks = 0; ks < kSteps; ++ks) {
+        const int k0 = (kq * kSteps + ks) * 16;
         uint32_t a0, a1, a2, a3;
         const int ar = mt * 16 + (lane & 15), ac = k0 + (lane >> 4) * 8;
         ldsm_x4(smem_u32(xh + ar * kXhStride + ac), a0, a1, a2, a3);
@@ -227,7 +232,7 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   }
 
   if constexpr (NT > 0) {
-    // fixed-order reduction of the four K quarters, then one bf16 rounding
+    // fixed-order reduction of the K parts, then one bf16 rounding
     const int mt = warp & 1, kq = warp >> 1;
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
@@ -245,9 +250,8 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       const int m = row0 + lr;
       if (m >= M || !ok) continue;
       float v = red[e];
-      v += red[kRows * kR + e];
-      v += red[2 * kRows * kR + e];
-      v += red[3 * kRows * kR + e];
+#pragma unroll
+      for (int part = 1; part < kKParts; ++part) v += red[part * kRows * kR + e];
       a.P[(size_t)m * kR + j] = (uint16_t)f32_to_bf16_bits(v);
     }
   }
@@ -270,12 +274,12 @@ cudaError_t launch_t(const QuantActArgs& a, unsigned* err, unsigned long long wa
     tm_l1 = tm_x;
   }
   const size_t smem = 1024 + (size_t)L::kStages * L::kStageBytes + (size_t)kRows * kXhStride * 2 +
-                      (NT ? (size_t)4 * kRows * kR * 4 : 0) + 64;
+                      (NT ? (size_t)kKParts * kRows * kR * 4 : 0) + 64;
   auto k = quant_act_kernel<PREC, NT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = (a.M + kRows - 1) / kRows;
-  k<<<grid, 256, smem, s>>>(tm_x, tm_l1, a, err, wait_ns);
+  k<<<grid, kThreadsQA, smem, s>>>(tm_x, tm_l1, a, err, wait_ns);
   return cudaGetLastError();
 }
 

@@ -145,6 +145,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// Bounded wait by a whole warp with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long ns, unsigned* err) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ns, err));
+}
+
 // --------------------------------------------------------------------------
 // TMA (tensor) and bulk copies
 // --------------------------------------------------------------------------

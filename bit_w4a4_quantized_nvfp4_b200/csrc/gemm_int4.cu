@@ -165,40 +165,55 @@ gemm_int4_kernel(const Params p) {
     }
   } else if (warp == kProdWarps) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks the loop and forms the descriptors; the elected
+    // lane issues the tcgen05 ops.
+    {
       uint32_t it = 0, gc = 0, tl = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tl) {
         for (int g = 0; g < p.NG; ++g, ++it, ++gc) {
           const int s = it % kStages;
           const int ab = gc & 1;
-          if (!mbar_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
-          if (!mbar_wait(&sm.acce[ab], ((gc >> 1) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
+          if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
+          if (!warp_wait(&sm.acce[ab], ((gc >> 1) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a = smem_u32(sm.a[s]), b = smem_u32(sm.b[s]);
+          uint64_t da[2], db[2];
 #pragma unroll
-          for (int k = 0; k < 2; ++k)
-            mma_i8(tmem + 128 * ab, make_sdesc(a + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone),
-                   make_sdesc(b + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone), kIdescI8, k ? 1u : 0u);
-          tc_commit(&sm.empty[s]);
-          tc_commit(&sm.accf[ab]);
+          for (int k = 0; k < 2; ++k) {
+            da[k] = make_sdesc(a + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone);
+            db[k] = make_sdesc(b + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone);
+          }
+          if (elect_one()) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) mma_i8(tmem + 128 * ab, da[k], db[k], kIdescI8, k ? 1u : 0u);
+            tc_commit(&sm.empty[s]);
+            tc_commit(&sm.accf[ab]);
+          }
+          __syncwarp();
         }
         if (!ok) break;
         if (has_lr) {
-          if (!mbar_wait(&sm.lr_full, tl & 1, p.wait_ns, p.err)) { ok = false; break; }
-          if (!mbar_wait(&sm.lr_acce, (tl & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
+          if (!warp_wait(&sm.lr_full, tl & 1, p.wait_ns, p.err)) { ok = false; break; }
+          if (!warp_wait(&sm.lr_acce, (tl & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t pa = smem_u32(sm.p), la = smem_u32(sm.l);
-          for (int k = 0; k < p.r / 16; ++k)
-            mma_bf16(tmem + kLrCol, make_sdesc(pa + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone),
-                     make_sdesc(la + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone), kIdescBf16,
-                     k ? 1u : 0u);
-          tc_commit(&sm.lr_empty);
-          tc_commit(&sm.lr_accf);
+          for (int k = 0; k < p.r / 16; ++k) {
+            const uint64_t da = make_sdesc(pa + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone);
+            const uint64_t db = make_sdesc(la + 2 * k * kChunkStride, kChunkStride, 128, kLayoutNone);
+            if (elect_one()) mma_bf16(tmem + kLrCol, da, db, kIdescBf16, k ? 1u : 0u);
+            __syncwarp();
+          }
+          if (elect_one()) {
+            tc_commit(&sm.lr_empty);
+            tc_commit(&sm.lr_accf);
+          }
+          __syncwarp();
         }
       }
-      tc_commit(&sm.mma_done);
-      (void)mbar_wait(&sm.mma_done, 0, p.wait_ns, p.err);
+      if (elect_one()) tc_commit(&sm.mma_done);
+      __syncwarp();
+      (void)warp_wait(&sm.mma_done, 0, p.wait_ns, p.err);
     }
   } else {
     // ------------------------------------------------------------ epilogue

@@ -76,11 +76,6 @@ struct Params {
   unsigned long long wait_ns;
 };
 
-// Bounded wait by a whole warp with a warp-uniform result.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long ns, unsigned* err) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ns, err));
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -189,22 +184,30 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
           const uint32_t st = smem_u32(sm.stage[s]);
           const uint32_t sfa = st + kABytes + kBBytes, sfb = sfa + kSfaBytes;
-          if (lane == 0) {
+          // Descriptors are formed by the whole warp (warp-uniform values) and
+          // the ops issued by the elected lane; building them inside a
+          // one-lane branch made every tcgen05 op markedly slower to issue.
+          uint64_t dcp[12], da[4], db[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            tc_cp_32x128b_warpx4_pair(tmem + kSfaCol + 4 * j, make_sdesc(sfa + 512 * j, 512, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4_pair(tmem + kSfbCol + 8 * j, make_sdesc(sfb + 512 * j, 512, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4_pair(tmem + kSfbCol + 8 * j + 4,
-                                      make_sdesc(sfb + 2048 + 512 * j, 512, 128, kLayoutNone));
+            dcp[3 * j] = make_sdesc(sfa + 512 * j, 512, 128, kLayoutNone);
+            dcp[3 * j + 1] = make_sdesc(sfb + 512 * j, 512, 128, kLayoutNone);
+            dcp[3 * j + 2] = make_sdesc(sfb + 2048 + 512 * j, 512, 128, kLayoutNone);
+            da[j] = make_sdesc(st + 32 * j, 16, 1024, kLayoutSw128);
+            db[j] = make_sdesc(st + kABytes + 32 * j, 16, 1024, kLayoutSw128);
           }
+          if (elect_one()) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t ad = make_sdesc(st + 32 * j, 16, 1024, kLayoutSw128);
-            const uint64_t bd = make_sdesc(st + kABytes + 32 * j, 16, 1024, kLayoutSw128);
-            mma_nvfp4_pair(acc, ad, bd, kIdescNvfp4, tmem + kSfaCol + 4 * j, tmem + kSfbCol + 8 * j,
-                           (kb > 0 || j > 0) ? 1u : 0u);
-          }
-          tc_commit_pair(&sm.empty[s], 0x3);
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_32x128b_warpx4_pair(tmem + kSfaCol + 4 * j, dcp[3 * j]);
+              tc_cp_32x128b_warpx4_pair(tmem + kSfbCol + 8 * j, dcp[3 * j + 1]);
+              tc_cp_32x128b_warpx4_pair(tmem + kSfbCol + 8 * j + 4, dcp[3 * j + 2]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              mma_nvfp4_pair(acc, da[j], db[j], kIdescNvfp4, tmem + kSfaCol + 4 * j, tmem + kSfbCol + 8 * j,
+                             (kb > 0 || j > 0) ? 1u : 0u);
+            tc_commit_pair(&sm.empty[s], 0x3);
           }
           __syncwarp();
         }
@@ -214,23 +217,22 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
           const uint32_t st = smem_u32(sm.stage[s]);
           const int half = p.r / 16;  // k16 steps per copy of P
-          if (lane == 0) {
-            for (int k = 0; k < 2 * half; ++k) {
-              const int kp = k % half;
-              const uint64_t ad = make_sdesc(st + 2 * kp * BM * 16, BM * 16, 128, kLayoutNone);
-              const uint64_t bd = make_sdesc(st + kABytes + 2 * k * BM * 16, BM * 16, 128, kLayoutNone);
-              mma_bf16_pair(acc, ad, bd, kIdescBf16, 1u);
-            }
-            tc_commit_pair(&sm.empty[s], 0x3);
+          for (int k = 0; k < 2 * half; ++k) {
+            const int kp = k % half;
+            const uint64_t ad = make_sdesc(st + 2 * kp * BM * 16, BM * 16, 128, kLayoutNone);
+            const uint64_t bd = make_sdesc(st + kABytes + 2 * k * BM * 16, BM * 16, 128, kLayoutNone);
+            if (elect_one()) mma_bf16_pair(acc, ad, bd, kIdescBf16, 1u);
+            __syncwarp();
           }
+          if (elect_one()) tc_commit_pair(&sm.empty[s], 0x3);
           __syncwarp();
           ++it;
         }
-        if (lane == 0) tc_commit_pair(&sm.acc_full[i & 1], 0x3);
+        if (elect_one()) tc_commit_pair(&sm.acc_full[i & 1], 0x3);
         __syncwarp();
       }
       // every MMA issued has completed before tensor memory is freed
-      if (lane == 0) tc_commit_pair(&sm.mma_done, 0x1);
+      if (elect_one()) tc_commit_pair(&sm.mma_done, 0x1);
       __syncwarp();
       (void)warp_wait(&sm.mma_done, 0, p.wait_ns, p.err);
     }

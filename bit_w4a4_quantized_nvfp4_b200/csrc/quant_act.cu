@@ -60,7 +60,8 @@ template <int NT>
 struct StageLayout {
   static constexpr int kR = NT * 8;
   static constexpr int kL1Bytes = NT ? kChunk * kR * 2 : 0;
-  static constexpr int kStageBytes = ((kXBytes + kL1Bytes + 1023) / 1024) * 1024;
+  static constexpr int kIlBytes = kChunk * 4;  // the chunk's inv_lambda
+  static constexpr int kStageBytes = ((kXBytes + kL1Bytes + kIlBytes + 1023) / 1024) * 1024;
   static constexpr int kStages = (kR <= 32) ? 4 : 3;
   // L1 tile rows are 2r bytes; the TMA swizzle span equals the row (32/64/128 B)
   static constexpr uint32_t kSwzMask = kR <= 16 ? 1u : (kR == 32 ? 3u : 7u);
@@ -79,8 +80,10 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = base;                                                      // S x kStageBytes
   __nv_bfloat16* xh = reinterpret_cast<__nv_bfloat16*>(base + S * L::kStageBytes);  // [32][264]
-  float* red = reinterpret_cast<float*>(xh + kRows * kXhStride);               // [kKParts][32][r]
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + (NT ? kKParts * kRows * kR : 0));
+  // [kKParts][32][r] partial P sums, written after the K loop when the stage
+  // buffers are idle (every issued stage has been consumed by then)
+  float* red = reinterpret_cast<float*>(stages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xh + kRows * kXhStride);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * kRows;
@@ -88,19 +91,20 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   const int nchunks = (K + kChunk - 1) / kChunk;
   const float s_tx = a.s_tx;
   const float six_t = __fmul_rn(6.0f, s_tx);
-  const uint32_t stage_tx = kXBytes + L::kL1Bytes;
+  auto issue_stage = [&](int c, uint8_t* st, uint64_t* bar) {
+    const int kcols = min(kChunk, K - c * kChunk);
+    mbar_expect_tx(bar, kXBytes + L::kL1Bytes + kcols * 4);
+    tma_load_2d(st, &tm_x, bar, c * kChunk, row0);
+    if (NT) tma_load_2d(st + kXBytes, &tm_l1, bar, 0, c * kChunk);
+    bulk_load(st + kXBytes + L::kL1Bytes, a.inv_lambda + (size_t)c * kChunk, (uint32_t)kcols * 4, bar);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     if (NT) tma_prefetch_desc(&tm_l1);
-    for (int c = 0; c < S && c < nchunks; ++c) {
-      uint8_t* st = stages + c * L::kStageBytes;
-      mbar_expect_tx(&full[c], stage_tx);
-      tma_load_2d(st, &tm_x, &full[c], c * kChunk, row0);
-      if (NT) tma_load_2d(st + kXBytes, &tm_l1, &full[c], 0, c * kChunk);
-    }
+    for (int c = 0; c < S && c < nchunks; ++c) issue_stage(c, stages + c * L::kStageBytes, &full[c]);
   }
   __syncthreads();
 
@@ -109,10 +113,14 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   for (int t = 0; t < (NT > 0 ? NT : 1); ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 
   bool ok = true;
+  int first_bad = nchunks;
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % S;
     uint8_t* st = stages + s * L::kStageBytes;
-    if (!mbar_wait(&full[s], (c / S) & 1, wait_ns, err)) ok = false;
+    if (ok && !mbar_wait(&full[s], (c / S) & 1, wait_ns, err)) {
+      ok = false;
+      first_bad = c;
+    }
     // every thread reaches the barriers below whatever happened, so that no
     // thread waits on one that others skipped
     const int col = c * kChunk + lane * 8;
@@ -120,8 +128,9 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
     float il[8];
     if (col_ok) {
-      const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + col));
-      const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.inv_lambda + col + 4));
+      const float* ils = reinterpret_cast<const float*>(st + kXBytes + L::kL1Bytes);
+      const float4 i0 = *reinterpret_cast<const float4*>(ils + lane * 8);
+      const float4 i1 = *reinterpret_cast<const float4*>(ils + lane * 8 + 4);
       il[0] = i0.x; il[1] = i0.y; il[2] = i0.z; il[3] = i0.w;
       il[4] = i1.x; il[5] = i1.y; il[6] = i1.z; il[7] = i1.w;
     } else {
@@ -224,13 +233,17 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
     __syncthreads();
     // stage s is free: refill it with chunk c + S
-    if (threadIdx.x == 0 && ok && c + S < nchunks) {
-      mbar_expect_tx(&full[s], stage_tx);
-      tma_load_2d(st, &tm_x, &full[s], (c + S) * kChunk, row0);
-      if (NT) tma_load_2d(st + kXBytes, &tm_l1, &full[s], 0, (c + S) * kChunk);
-    }
+    if (threadIdx.x == 0 && ok && c + S < nchunks) issue_stage(c + S, st, &full[s]);
   }
 
+  if (!ok) {
+    // a stage never completed: let the copies already issued land before the
+    // CTA exits (bounded), and write nothing more
+    if (threadIdx.x == 0)
+      for (int c = first_bad; c < nchunks && c < first_bad + S; ++c)
+        (void)mbar_wait(&full[c % S], (c / S) & 1, wait_ns, nullptr);
+    return;
+  }
   if constexpr (NT > 0) {
     // fixed-order reduction of the K parts, then one bf16 rounding
     const int mt = warp & 1, kq = warp >> 1;
@@ -273,8 +286,8 @@ cudaError_t launch_t(const QuantActArgs& a, unsigned* err, unsigned long long wa
   } else {
     tm_l1 = tm_x;
   }
-  const size_t smem = 1024 + (size_t)L::kStages * L::kStageBytes + (size_t)kRows * kXhStride * 2 +
-                      (NT ? (size_t)kKParts * kRows * kR * 4 : 0) + 64;
+  static_assert((size_t)kKParts * kRows * kR * 4 <= (size_t)L::kStages * L::kStageBytes, "reduction fits the stages");
+  const size_t smem = 1024 + (size_t)L::kStages * L::kStageBytes + (size_t)kRows * kXhStride * 2 + 64;
   auto k = quant_act_kernel<PREC, NT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

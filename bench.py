@@ -21,11 +21,17 @@ is the maximum over ranks.
 
 ``--impl reference`` times the CPU oracle (the only reference implementation
 of this path) on a bounded row sample of the same workload.
+
+Roofline traffic: DRAM bytes per launch of the GEMM kernel as read by one
+`ncu --set full` capture (dram__bytes_read.sum + dram__bytes_write.sum). The
+figure is tied to the SHA-256 of the kernel source it was taken on and is
+reported as null once that source has changed.
 """
 
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -47,6 +53,18 @@ METRIC = "SVDQ W4A4-NVFP4 linear TFLOPS, % dense FP4 peak (M4608 K3072 N9216 r32
 FP4_DENSE_SPEC_TFLOPS = 9000.0
 NOMINAL_FP4_OVER_BF16 = 4.0     # 9 PF / 2.25 PF dense
 L2_FLUSH_BYTES = 512 << 20
+GEMM_SOURCE = os.path.join(ROOT, "bit_w4a4_quantized_nvfp4_b200", "csrc", "gemm_nvfp4.cu")
+# {sha256 of the GEMM kernel source: DRAM bytes per launch from an ncu capture of the workload}
+GEMM_TRAFFIC = {}
+
+
+def gemm_traffic():
+    try:
+        with open(GEMM_SOURCE, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return GEMM_TRAFFIC.get(digest)
 
 
 def peaks():
@@ -115,18 +133,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, timeout_s: float = 120.0):
+    """Join the torchrun job (one rank per GPU, NCCL); without a GPU the same
+    host logic runs over gloo (used by the CPU tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if world > 1:
         import datetime
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
+        if cuda:
+            torch.cuda.set_device(local)
+        dist.init_process_group("nccl" if cuda else "gloo", timeout=datetime.timedelta(seconds=timeout_s))
+    elif cuda:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -143,9 +165,16 @@ def max_over_ranks(world, v: float) -> float:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Throughput of all ranks together: every rank runs one step of the same
+    size, and the step time is the slowest rank's."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
 
 
 def bf16_dev(bits):
@@ -214,7 +243,7 @@ def run_cuda(args):
     k1 = max_over_ranks(world, statistics.mean(k1_ms))
     k2 = max_over_ranks(world, statistics.mean(k2_ms))
     flops = 2.0 * M * N * K
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, ms)
 
     # end to end through the public API with host buffers
     xh = torch.from_numpy(np.ascontiguousarray(d["x"]).view(np.int16)).pin_memory()
@@ -265,8 +294,8 @@ def run_cuda(args):
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(k2_tflops / fp4_peak, 4),
                      "peak_source": f"{P['source']} bf16 burst {P['bf16']} x nominal fp4/bf16 ratio 4",
-                     "traffic": None},
-        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+                     "traffic": gemm_traffic()},
+        "e2e": {"value": round(whole_job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
         "gpu_launches": 2 * K_steps,
         "wall_s_timed_region": round(wall, 4),
@@ -328,8 +357,8 @@ def cpu_baseline(d, rows: int, tag="oracle"):
     oracle.linear("nvfp4", a, w, 1.0, d["L2"], d["b"])
     dt = time.perf_counter() - t0
     return {"value": round(2.0 * rows * N * K / dt / 1e12, 6), "unit": "TFLOPS", "cores": oracle.threads(),
-            "kind": tag, "sample": f"first {rows} of {c['M']} rows of the workload (quantize_act + linear, "
-                                    "float64 accumulation); weight pack untimed", "seconds": round(dt, 3)}
+            "kind": tag, "sample": f"first {min(rows, c['M'])} of {c['M']} rows of the workload (quantize_act + "
+                                    "linear, float64 accumulation); weight pack untimed", "seconds": round(dt, 3)}
 
 
 def run_reference(args):
@@ -375,7 +404,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--cpu-rows", type=int, default=4608)
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-awq", action="store_true")

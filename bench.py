@@ -55,7 +55,10 @@ NOMINAL_FP4_OVER_BF16 = 4.0     # 9 PF / 2.25 PF dense
 L2_FLUSH_BYTES = 512 << 20
 GEMM_SOURCE = os.path.join(ROOT, "bit_w4a4_quantized_nvfp4_b200", "csrc", "gemm_nvfp4.cu")
 # {sha256 of the GEMM kernel source: DRAM bytes per launch from an ncu capture of the workload}
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {
+    # profiles/gemm_nvfp4_c3.md: 25,487,616 B read + 32,836,352 B written
+    "690fa580dee2e9d705b7229094317cd847e605a334b36eea882d3d683c685fe5": 58323968,
+}
 
 
 def gemm_traffic():

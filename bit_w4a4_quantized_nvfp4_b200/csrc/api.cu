@@ -235,10 +235,11 @@ svdq_status awq_w4a16_linear(int M, int K, int N, const uint16_t* x, const uint8
   if (!aligned16(x) || !aligned16(q) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y) ||
       (bias && (reinterpret_cast<uintptr_t>(bias) & 1)))
     return SVDQ_ERR_ALIGN;
-  svdq_status st = device_info(nullptr, nullptr);
+  unsigned* err = nullptr;
+  svdq_status st = device_info(&err, nullptr);
   if (st != SVDQ_OK) return st;
   AwqArgs a{x, q, scales, zeros, bias, y, M, K, N};
-  return from_cuda(launch_awq(a, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_awq(a, err, g_wait_ns.load(), static_cast<cudaStream_t>(stream)));
 }
 
 svdq_status svdq_device_error(unsigned* bits) {

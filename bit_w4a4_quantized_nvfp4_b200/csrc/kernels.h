@@ -54,7 +54,7 @@ struct AwqArgs {
   uint16_t* y;
   int M, K, N;
 };
-cudaError_t launch_awq(const AwqArgs& a, cudaStream_t s);
+cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 
 struct GemmArgs {
   const uint8_t* x_codes;

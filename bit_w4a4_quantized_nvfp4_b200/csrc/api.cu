@@ -229,7 +229,7 @@ svdq_status awq_pack_weight(int K, int N, const float* W, uint8_t* q, uint16_t* 
 svdq_status awq_w4a16_linear(int M, int K, int N, const uint16_t* x, const uint8_t* q, const uint16_t* scales,
                              const uint16_t* zeros, const uint16_t* bias, uint16_t* y, void* stream) {
   if (M < 0 || K <= 0 || N <= 0) return SVDQ_ERR_INVALID_ARG;
-  if (K % 64 || N % 8) return SVDQ_ERR_SHAPE;
+  if (K % 64 || N % 8 || K > 16384) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!x || !q || !scales || !zeros || !y) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(q) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y) ||

@@ -11,6 +11,11 @@
 // two warp groups take alternate stages, so a stage is only refilled for the
 // group that released it).
 //
+// The CTA's activations (up to 16 rows) and its rows' group scales and zero
+// points (one contiguous range each) are copied into shared memory once, at
+// the start, by bulk copies; the activations are then permuted in place into MMA-fragment order
+// so that the inner loop reads each B fragment with one 16-byte load.
+//
 // Compute warp (row tile rt of 16 weight rows, stage phase kh): per 64-group
 // it unpacks its two rows' nibbles to bf16 with bit operations ((128 + q) has
 // an exact bf16 encoding; subtracting 128 + z leaves q - z exactly) and lets
@@ -21,9 +26,9 @@
 // K order inside a group: lane t of a row quad owns k = 16t .. 16t+15 (one
 // 8-byte shared load per row). Its nibbles are used in pairs (k, k+4), fed to
 // the MMA K slots in the order (0,4),(1,5) | (2,6),(3,7) | (8,12),(9,13) |
-// (10,14),(11,15) for the four k16 steps; the activation fragments are built
-// in the same order from two 16-byte loads of x, so the dot product is
-// unchanged.
+// (10,14),(11,15) for the four k16 steps; each 16-element block of x is
+// stored as the bf16 pairs (0,4) (1,5) (2,6) (3,7) (8,12) (9,13) (10,14)
+// (11,15), so the dot product is unchanged.
 #include "device.cuh"
 #include "kernels.h"
 
@@ -33,10 +38,11 @@ namespace {
 constexpr int kRowsA = 64;                          // weight rows (output columns) per CTA
 constexpr int kStageK = 256;                        // K per stage: 4 groups, 128 bytes per row
 constexpr int kStageBytesA = kRowsA * kStageK / 2;  // 8 KB
-constexpr int kStagesA = 8;                         // even: see the header comment
+constexpr int kStagesA = 6;                         // even: see the header comment
 constexpr int kComputeWarps = 8;                    // 4 row tiles x 2 stage phases
 constexpr int kThreadsA = (kComputeWarps + 1) * 32;
 constexpr int kMaxM = 16;                           // batch rows per launch (two m-tiles of 8)
+constexpr int kAwqSmemLimit = 232448;               // dynamic shared memory per CTA on sm_100
 static_assert(kStagesA % 2 == 0, "a stage is reused by one warp group only");
 
 __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -62,29 +68,49 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
-struct SmemA {
-  uint8_t stage[kStagesA][kStageBytesA];  // 1024-aligned
-  float red[4][2][32][4];                 // phase-1 partial sums [rt][mt][lane][c]
-  uint64_t full[kStagesA], empty[kStagesA];
-  int abort_flag;
+// Shared-memory plan of one CTA (dynamic size: it depends on M and K).
+struct AwqLayout {
+  int x_pitch;    // bytes per activation row: 2K + 16 (the pad spreads rows over banks)
+  int sz_pitch;   // bytes per weight row of scales / zeros: 2 * (K / 64)
+  int off_x, off_s, off_z, off_bar, total;
+  __host__ __device__ AwqLayout(int M, int K) {
+    const int ng = K / 64;
+    x_pitch = 2 * K + 16;
+    sz_pitch = 2 * ng;
+    off_x = kStagesA * kStageBytesA;
+    off_s = off_x + M * x_pitch;
+    off_z = ((off_s + kRowsA * sz_pitch + 15) / 16) * 16;
+    off_bar = ((off_z + kRowsA * sz_pitch + 15) / 16) * 16;
+    total = off_bar + 2 * kStagesA * 8 + 8 + 16 + 4 * 2 * 32 * 4 * 4;
+  }
 };
 
 __global__ void __launch_bounds__(kThreadsA, 2)
 awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
-  SmemA& sm = *reinterpret_cast<SmemA*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = a.K, N = a.N, M = a.M;
   const int ng = K / 64;
   const int nst = (K + kStageK - 1) / kStageK;
   const int n0 = blockIdx.x * kRowsA;
+  const AwqLayout L(M, K);
+  uint8_t* xs = base + L.off_x;
+  const uint8_t* ss = base + L.off_s;
+  const uint8_t* zs = base + L.off_z;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + L.off_bar);
+  uint64_t* empty = full + kStagesA;
+  uint64_t* xbar = empty + kStagesA;
+  int* abort_flag = reinterpret_cast<int*>(xbar + 1);
+  float* red = reinterpret_cast<float*>(abort_flag + 4);  // phase-1 partial sums [rt][mt][lane][4]
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesA; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 4);
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
     }
-    sm.abort_flag = 0;
+    mbar_init(xbar, 1);
+    *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -93,71 +119,87 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
+      // activations (one bulk copy per row) and this CTA's rows of scales and
+      // zero points (contiguous: rows n0 .. n0 + rows - 1, 16-byte aligned)
+      const uint32_t sz_bytes = (uint32_t)(min(kRowsA, N - n0) * L.sz_pitch);
+      mbar_expect_tx(xbar, (uint32_t)(M * 2 * K) + 2 * sz_bytes);
+      for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
+      bulk_load(base + L.off_s, a.s + (size_t)n0 * ng, sz_bytes, xbar);
+      bulk_load(base + L.off_z, a.z + (size_t)n0 * ng, sz_bytes, xbar);
       int c = 0;
       bool ok = true;
       for (; c < nst; ++c) {
         const int s = c % kStagesA;
-        if (c >= kStagesA && !mbar_wait(&sm.empty[s], ((c / kStagesA) - 1) & 1, wait_ns, err)) {
+        if (c >= kStagesA && !mbar_wait(&empty[s], ((c / kStagesA) - 1) & 1, wait_ns, err)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(&sm.full[s], kStageBytesA);
-        tma_load_2d(sm.stage[s], &tm_q, &sm.full[s], c * (kStageK / 2), n0);
+        uint8_t* st = base + s * kStageBytesA;
+        mbar_expect_tx(&full[s], kStageBytesA);
+        tma_load_2d(st, &tm_q, &full[s], c * (kStageK / 2), n0);
       }
-      if (!ok) {
-        // let the copies already issued land before the CTA can exit (bounded)
+      // let the copies already issued land before the CTA can exit (bounded)
+      (void)mbar_wait(xbar, 0, wait_ns, ok ? err : nullptr);
+      if (!ok)
         for (int j = max(0, c - kStagesA); j < c; ++j)
-          (void)mbar_wait(&sm.full[j % kStagesA], (j / kStagesA) & 1, wait_ns, nullptr);
-      }
+          (void)mbar_wait(&full[j % kStagesA], (j / kStagesA) & 1, wait_ns, nullptr);
     }
     return;
   }
 
   // ---------------------------------------------------------------- compute
+  bool ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0, wait_ns, err));
+  // permute every 16-element block of x in place into fragment-pair order
+  if (ok) {
+    const int blocks = M * (K / 16);
+    for (int b = threadIdx.x; b < blocks; b += kComputeWarps * 32) {
+      const int m = b / (K / 16), kb = b % (K / 16);
+      uint4* p = reinterpret_cast<uint4*>(xs + m * L.x_pitch + kb * 32);
+      const uint4 u = p[0], v = p[1];
+      p[0] = make_uint4(prmt(u.x, u.z, 0x5410u), prmt(u.x, u.z, 0x7632u), prmt(u.y, u.w, 0x5410u),
+                        prmt(u.y, u.w, 0x7632u));
+      p[1] = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u), prmt(v.y, v.w, 0x5410u),
+                        prmt(v.y, v.w, 0x7632u));
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarps * 32) : "memory");
+
   const int rt = warp & 3, kh = warp >> 2;
   const int gid = lane >> 2, t = lane & 3;
   const int r_lo = rt * 16 + gid, r_hi = r_lo + 8;  // rows within the CTA's 64
   const int n_lo = n0 + r_lo, n_hi = n0 + r_hi;
   const bool ok_lo = n_lo < N, ok_hi = n_hi < N;
   const int mt_count = (M + 7) / 8;
-  // batch rows of this lane's B fragments (column gid of each m-tile)
-  const uint16_t* x0 = gid < M ? a.x + (size_t)gid * K + 16 * t : nullptr;
-  const uint16_t* x1 = gid + 8 < M ? a.x + (size_t)(gid + 8) * K + 16 * t : nullptr;
-  const uint16_t* s_lo = a.s + (size_t)(ok_lo ? n_lo : 0) * ng;
-  const uint16_t* s_hi = a.s + (size_t)(ok_hi ? n_hi : 0) * ng;
-  const uint16_t* z_lo = a.z + (size_t)(ok_lo ? n_lo : 0) * ng;
-  const uint16_t* z_hi = a.z + (size_t)(ok_hi ? n_hi : 0) * ng;
+  // this lane's B-fragment rows (column gid of each m-tile), 16t into each group
+  const uint8_t* x0 = gid < M ? xs + gid * L.x_pitch + 32 * t : nullptr;
+  const uint8_t* x1 = gid + 8 < M ? xs + (gid + 8) * L.x_pitch + 32 * t : nullptr;
 
   float tot[2][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i) tot[i][0] = tot[i][1] = tot[i][2] = tot[i][3] = 0.f;
 
-  bool ok = true;
-  for (int c = kh; c < nst; c += 2) {
+  for (int c = kh; c < nst && ok; c += 2) {
     const int s = c % kStagesA;
-    // this stage's group scales and zero points (issued before the wait)
     const int g0 = c * 4, gn = min(4, ng - g0);
-    uint32_t sv[4], zv[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int g = min(g0 + j, ng - 1);
-      sv[j] = (uint32_t)__ldg(s_lo + g) | ((uint32_t)__ldg(s_hi + g) << 16);
-      zv[j] = (uint32_t)__ldg(z_lo + g) | ((uint32_t)__ldg(z_hi + g) << 16);
-    }
-    if (!warp_wait(&sm.full[s], (c / kStagesA) & 1, wait_ns, err)) {
+    if (!warp_wait(&full[s], (c / kStagesA) & 1, wait_ns, err)) {
       ok = false;
       break;
     }
-    const uint8_t* st = sm.stage[s];
+    const uint8_t* st = base + s * kStageBytesA;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       if (j < gn) {
+        const int g = g0 + j;
         // weights: 8 bytes of rows r_lo and r_hi (group j, k = 16t ..), 128-byte swizzle
         const int u = 2 * j + (t >> 1), hoff = (t & 1) * 8;
         const uint2 wl = *reinterpret_cast<const uint2*>(st + r_lo * 128 + ((u ^ (r_lo & 7)) << 4) + hoff);
         const uint2 wh = *reinterpret_cast<const uint2*>(st + r_hi * 128 + ((u ^ (r_hi & 7)) << 4) + hoff);
-        const uint32_t zzl = f32_to_bf16_bits(128.0f + bf16_bits_to_f32(zv[j] & 0xFFFFu)) * 0x10001u;
-        const uint32_t zzh = f32_to_bf16_bits(128.0f + bf16_bits_to_f32(zv[j] >> 16)) * 0x10001u;
+        const uint32_t zl = *reinterpret_cast<const uint16_t*>(zs + r_lo * L.sz_pitch + 2 * g);
+        const uint32_t zh = *reinterpret_cast<const uint16_t*>(zs + r_hi * L.sz_pitch + 2 * g);
+        const float sc_lo = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + r_lo * L.sz_pitch + 2 * g));
+        const float sc_hi = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(ss + r_hi * L.sz_pitch + 2 * g));
+        const uint32_t zzl = f32_to_bf16_bits(128.0f + bf16_bits_to_f32(zl)) * 0x10001u;
+        const uint32_t zzh = f32_to_bf16_bits(128.0f + bf16_bits_to_f32(zh)) * 0x10001u;
         uint32_t A[4][4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -169,25 +211,20 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
           A[q][2] = deq_pair(wlo, sh0 + 4, zzl);
           A[q][3] = deq_pair(whi, sh0 + 4, zzh);
         }
-        const float sc_lo = bf16_bits_to_f32(sv[j] & 0xFFFFu), sc_hi = bf16_bits_to_f32(sv[j] >> 16);
-        const int kof = (g0 + j) * 64;
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
           if (mt < mt_count) {
-            const uint16_t* xp = mt ? x1 : x0;
+            const uint8_t* xp = mt ? x1 : x0;
             uint4 xa = make_uint4(0, 0, 0, 0), xb = make_uint4(0, 0, 0, 0);
             if (xp) {
-              xa = __ldg(reinterpret_cast<const uint4*>(xp + kof));
-              xb = __ldg(reinterpret_cast<const uint4*>(xp + kof + 8));
+              xa = *reinterpret_cast<const uint4*>(xp + 128 * g);
+              xb = *reinterpret_cast<const uint4*>(xp + 128 * g + 16);
             }
-            // pairs (k, k+4): (0,4) (1,5) | (2,6) (3,7) | (8,12) (9,13) | (10,14) (11,15)
-            const uint32_t B[4][2] = {{prmt(xa.x, xa.z, 0x5410u), prmt(xa.x, xa.z, 0x7632u)},
-                                      {prmt(xa.y, xa.w, 0x5410u), prmt(xa.y, xa.w, 0x7632u)},
-                                      {prmt(xb.x, xb.z, 0x5410u), prmt(xb.x, xb.z, 0x7632u)},
-                                      {prmt(xb.y, xb.w, 0x5410u), prmt(xb.y, xb.w, 0x7632u)}};
             float cc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) mma_16816(cc, A[q], B[q][0], B[q][1]);
+            mma_16816(cc, A[0], xa.x, xa.y);
+            mma_16816(cc, A[1], xa.z, xa.w);
+            mma_16816(cc, A[2], xb.x, xb.y);
+            mma_16816(cc, A[3], xb.z, xb.w);
             tot[mt][0] = fmaf(sc_lo, cc[0], tot[mt][0]);
             tot[mt][1] = fmaf(sc_lo, cc[1], tot[mt][1]);
             tot[mt][2] = fmaf(sc_hi, cc[2], tot[mt][2]);
@@ -197,19 +234,20 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.empty[s]);
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 
   // add the two phases' partial sums (phase 0 + phase 1) and store
-  if (!ok && lane == 0) sm.abort_flag = 1;
+  if (!ok && lane == 0) *abort_flag = 1;
+  float* rb = red + (size_t)rt * 2 * 32 * 4;
   if (kh == 1) {
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sm.red[rt][mt][lane][i] = tot[mt][i];
+      for (int i = 0; i < 4; ++i) rb[(mt * 32 + lane) * 4 + i] = tot[mt][i];
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarps * 32) : "memory");
-  if (sm.abort_flag || kh == 1) return;
+  if (*abort_flag || kh == 1) return;
   const float b_lo = (a.bias && ok_lo) ? bf16_bits_to_f32(a.bias[n_lo]) : 0.f;
   const float b_hi = (a.bias && ok_hi) ? bf16_bits_to_f32(a.bias[n_hi]) : 0.f;
 #pragma unroll
@@ -219,8 +257,8 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
     for (int i = 0; i < 2; ++i) {
       const int m = mt * 8 + 2 * t + i;  // column 2t + i of the MMA tile
       if (m >= M) continue;
-      const float v_lo = tot[mt][i] + sm.red[rt][mt][lane][i];
-      const float v_hi = tot[mt][2 + i] + sm.red[rt][mt][lane][2 + i];
+      const float v_lo = tot[mt][i] + rb[(mt * 32 + lane) * 4 + i];
+      const float v_hi = tot[mt][2 + i] + rb[(mt * 32 + lane) * 4 + 2 + i];
       if (ok_lo) a.y[(size_t)m * N + n_lo] = (uint16_t)f32_to_bf16_bits(__fadd_rn(v_lo, b_lo));
       if (ok_hi) a.y[(size_t)m * N + n_hi] = (uint16_t)f32_to_bf16_bits(__fadd_rn(v_hi, b_hi));
     }
@@ -229,21 +267,30 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
 
 }  // namespace
 
+int awq_rows_per_launch(int K) {
+  // as many batch rows (up to 16) as leave the CTA's shared memory within bounds
+  int mb = kMaxM;
+  while (mb > 0 && AwqLayout(mb, K).total + 1024 > kAwqSmemLimit) --mb;
+  return mb;
+}
+
 cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s) {
   CUtensorMap tm_q;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q, (uint64_t)a.K / 2, (uint64_t)a.N, (uint64_t)a.K / 2,
                     kStageK / 2, kRowsA, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const size_t smem = sizeof(SmemA) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(awq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  const int mb = awq_rows_per_launch(a.K);
+  if (mb < 1) return cudaErrorInvalidValue;
   const int grid = (a.N + kRowsA - 1) / kRowsA;
-  // batch rows are taken 16 at a time; each block of rows re-reads the weights
-  for (int m0 = 0; m0 < a.M; m0 += kMaxM) {
+  // batch rows are taken mb at a time; each block of rows re-reads the weights
+  for (int m0 = 0; m0 < a.M; m0 += mb) {
     AwqArgs b = a;
-    b.M = min(kMaxM, a.M - m0);
+    b.M = min(mb, a.M - m0);
     b.x = a.x + (size_t)m0 * a.K;
     b.y = a.y + (size_t)m0 * a.N;
+    const size_t smem = (size_t)AwqLayout(b.M, a.K).total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(awq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     awq_kernel<<<grid, kThreadsA, smem, s>>>(tm_q, b, err, wait_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

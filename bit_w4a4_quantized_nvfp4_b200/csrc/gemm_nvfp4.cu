@@ -22,14 +22,18 @@
 //               (into both CTAs' tensor memory) and 4 x tcgen05.mma
 //               kind::mxf4nvf4 (K = 64); after the K loop, tcgen05.mma
 //               kind::f16 adds P (hi + lo) into the same accumulator.
-//   warps 2..5  epilogue (both CTAs): tcgen05.ld, y = alpha*acc + bias,
-//               convert, stage a whole 128 x 256 output tile in 128B-swizzled
-//               shared memory, TMA store.
+//   warps 2..9  epilogue (both CTAs), two warps per TMEM lane quadrant, each
+//               draining half of the 256 columns: tcgen05.ld, y = alpha*acc +
+//               bias, convert, stage 32 x 64 pieces in 128B-swizzled shared
+//               memory, TMA store.
 // Accumulators: two 256-column buffers overlapping in 64 columns
-// ([0,256) and [192,448); scales in [448,512)). The epilogue drains the
-// overlapped 64 columns first and releases them, so the next tile's MMAs
-// start after a quarter of the drain; the output tile's stores run under the
-// next tile's mainloop. Every mbarrier wait is bounded in wall time.
+// ([0,256) and [192,448); scales in [448,512)). Per tile, the epilogue half
+// that holds the overlapped 64 columns drains them first and then releases
+// the tile; the other half releases it as soon as it has finished the
+// previous tile. The next tile's MMAs therefore start after an eighth of the
+// drain, and the output stores run under the next tile's mainloop. One
+// release barrier per accumulator buffer keeps the arrivals of consecutive
+// tiles apart. Every mbarrier wait is bounded in wall time.
 #include "device.cuh"
 #include "kernels.h"
 
@@ -44,9 +48,9 @@ constexpr int kSfaBytes = 4 * 512;              // 4 K-atoms x 128 rows
 constexpr int kSfbBytes = 2 * 4 * 512;          // the pair's 256 N rows x 4 K-atoms (both CTAs)
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr uint32_t kStageTx = 2u * kStageBytes;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;
 constexpr int kSlotBytes = 32 * 128;            // 32 rows x 128 bytes (one TMA store box)
-constexpr int kSlots = 4;
+constexpr int kSlots = 2;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol0 = 0, kAccCol1 = 192;
@@ -59,9 +63,9 @@ constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
 struct Smem {
   uint8_t stage[kStages][kStageBytes];          // 1024-aligned (kStageBytes % 1024 == 0)
   uint8_t out[kEpiWarps][kSlots][kSlotBytes];
-  float bias[kEpiWarps][BN];
+  float bias[kEpiWarps][BN / 2];
   uint64_t full[kStages], empty[kStages];
-  uint64_t acc_full[2], acc_free, mma_done;
+  uint64_t acc_full[2], acc_free[2], mma_done;
   uint32_t tmem_base;
 };
 static_assert(kStageBytes % 1024 == 0, "stage alignment");
@@ -98,7 +102,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     }
     mbar_init(&sm.acc_full[0], 1);
     mbar_init(&sm.acc_full[1], 1);
-    mbar_init(&sm.acc_free, 2 * kEpiWarps);
+    mbar_init(&sm.acc_free[0], 2 * kEpiWarps);
+    mbar_init(&sm.acc_free[1], 2 * kEpiWarps);
     mbar_init(&sm.mma_done, 1);
     fence_mbar_init();
   }
@@ -174,7 +179,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       int i = 0;
       for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++i) {
         const uint32_t acc = tmem + ((i & 1) ? kAccCol1 : kAccCol0);
-        if (i > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(&sm.acc_free, (i - 1) & 1, p.wait_ns, p.err))) {
+        // tile i - 1 released: its overlapped columns are drained and tile
+        // i - 2 (the previous user of this buffer) is drained completely
+        if (i > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(&sm.acc_free[(i - 1) & 1], ((i - 1) >> 1) & 1,
+                                                                 p.wait_ns, p.err))) {
           ok = false;
           break;
         }
@@ -240,37 +248,45 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quadrant of this warp
     const int e = warp - 2;              // epilogue warp index (staging slots)
+    const int h = e >> 2;                // column half: [128 h, 128 h + 128)
     const float alpha = __fmul_rn(p.tensor_scale[0], p.tensor_scale[1]);
-    const uint32_t free_bar = mapa_shared(smem_u32(&sm.acc_free), 0);
     const int cols = p.out_f32 ? 32 : 64;          // columns per chunk
-    const int nchunks = BN / cols;
-    const int release_after = 64 / cols - 1;       // chunks covering the 64 overlapped columns
+    const int nchunks = (BN / 2) / cols;           // chunks per half
+    const int overlap_chunks = 64 / cols;          // chunks covering the 64 shared columns
     float* bias = sm.bias[e];
     int i = 0;
     for (int tile = pair; tile < num_tiles; tile += npairs, ++i) {
       const int tm = tile / p.tiles_n, tn = tile % p.tiles_n;
       const int row0 = tm * 256 + (int)rank * BM + 32 * q;
-      const int n0 = tn * BN;
+      const int n0 = tn * BN + 128 * h;
       const int b = i & 1;
+      // buffer 0 shares its top 64 columns (half 1), buffer 1 its bottom 64 (half 0)
+      const bool holds_overlap = (b == 0) == (h == 1);
+      const uint32_t free_bar = mapa_shared(smem_u32(&sm.acc_free[b]), 0);
       __syncwarp();
-      for (int c = lane; c < BN; c += 32) {
+      for (int c = lane; c < BN / 2; c += 32) {
         const int n = n0 + c;
         bias[c] = (p.bias && n < p.N) ? bf16_bits_to_f32(p.bias[n]) : 0.f;
       }
       __syncwarp();
+      if (!holds_overlap) {
+        // this warp is done with the previous tile: release this one for it
+        tc_fence_before();
+        if (lane == 0) mbar_arrive_cluster(free_bar);
+      }
       if (!mbar_wait(&sm.acc_full[b], (i >> 1) & 1, p.wait_ns, p.err)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + (b ? kAccCol1 : kAccCol0) + ((uint32_t)(32 * q) << 16);
+      const uint32_t tbase = tmem + (b ? kAccCol1 : kAccCol0) + 128 * h + ((uint32_t)(32 * q) << 16);
       for (int step = 0; step < nchunks; ++step) {
-        // buffer 0 drains from its high end, buffer 1 from its low end: both
-        // start with the columns the other buffer shares
-        const int c = b == 0 ? nchunks - 1 - step : step;
+        // buffer 0's upper half drains from its top, everything else from the
+        // bottom: the shared columns come first
+        const int c = (b == 0 && h == 1) ? nchunks - 1 - step : step;
         uint8_t* buf = sm.out[e][step % kSlots];
         uint32_t v[32], v2[32];
         tmem_ld32(tbase + cols * c, v);
         if (!p.out_f32) tmem_ld32(tbase + cols * c + 32, v2);
         tmem_ld_wait();
-        if (step == release_after) {
+        if (holds_overlap && step == overlap_chunks - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(free_bar);
@@ -280,22 +296,27 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (p.out_f32) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            float o[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] = fmaf(alpha, __uint_as_float(v[4 * u + k]), bias[32 * c + 4 * u + k]);
-            *reinterpret_cast<float4*>(buf + lane * 128 + ((u ^ (lane & 7)) * 16)) = make_float4(o[0], o[1], o[2], o[3]);
+            const float4 bv = *reinterpret_cast<const float4*>(bias + 32 * c + 4 * u);
+            const float o0 = fmaf(alpha, __uint_as_float(v[4 * u]), bv.x);
+            const float o1 = fmaf(alpha, __uint_as_float(v[4 * u + 1]), bv.y);
+            const float o2 = fmaf(alpha, __uint_as_float(v[4 * u + 2]), bv.z);
+            const float o3 = fmaf(alpha, __uint_as_float(v[4 * u + 3]), bv.w);
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((u ^ (lane & 7)) * 16)) = make_float4(o0, o1, o2, o3);
           }
         } else {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
+            const float4 b0 = *reinterpret_cast<const float4*>(bias + 64 * c + 8 * u);
+            const float4 b1 = *reinterpret_cast<const float4*>(bias + 64 * c + 8 * u + 4);
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
             uint32_t w4[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int col = 8 * u + 2 * k;
               const uint32_t a0 = col < 32 ? v[col] : v2[col - 32];
               const uint32_t a1 = col + 1 < 32 ? v[col + 1] : v2[col + 1 - 32];
-              const float y0 = fmaf(alpha, __uint_as_float(a0), bias[64 * c + col]);
-              const float y1 = fmaf(alpha, __uint_as_float(a1), bias[64 * c + col + 1]);
+              const float y0 = fmaf(alpha, __uint_as_float(a0), bb[2 * k]);
+              const float y1 = fmaf(alpha, __uint_as_float(a1), bb[2 * k + 1]);
               w4[k] = f32_to_bf16_bits(y0) | (f32_to_bf16_bits(y1) << 16);
             }
             *reinterpret_cast<uint4*>(buf + lane * 128 + ((u ^ (lane & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);

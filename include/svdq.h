@@ -160,7 +160,8 @@ svdq_status awq_pack_weight(int K, int N, const float* W, uint8_t* q, uint16_t* 
  *   y[m,n] = bf16( sum_g s[n,g] sum_{k in g} x[m,k] (q[n,k] - z[n,g]) + bias[n] )
  * In:  x bf16 [M, K]; q, scales, zeros from awq_pack_weight; bias bf16 [N] or NULL.
  * Out: y bf16 [M, N].
- * Shapes: K % 64 == 0, N % 8 == 0, M >= 0. */
+ * Shapes: K % 64 == 0, K <= 16384 (the activations of a block of rows are
+ * held in shared memory), N % 8 == 0, M >= 0. */
 svdq_status awq_w4a16_linear(int M, int K, int N, const uint16_t* x, const uint8_t* q,
                              const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias,
                              uint16_t* y, void* stream);

@@ -24,8 +24,8 @@
 //               kind::f16 adds P (hi + lo) into the same accumulator.
 //   warps 2..9  epilogue (both CTAs), two warps per TMEM lane quadrant, each
 //               draining half of the 256 columns: tcgen05.ld, y = alpha*acc +
-//               bias, convert, stage 32 x 64 pieces in 128B-swizzled shared
-//               memory, TMA store.
+//               bias (read through the L1 cache), convert, stage 32 x 64
+//               pieces in 128B-swizzled shared memory, TMA store.
 // Accumulators: two 256-column buffers overlapping in 64 columns
 // ([0,256) and [192,448); scales in [448,512)). Per tile, the epilogue half
 // that holds the overlapped 64 columns drains them first and then releases
@@ -41,7 +41,7 @@ namespace svdq {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;    // per-CTA rows, pair N, K per stage (FP4 elements)
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kABytes = BM * BK / 2;            // 16 KB
 constexpr int kBBytes = (BN / 2) * BK / 2;      // 16 KB (this CTA's half of the N tile)
 constexpr int kSfaBytes = 4 * 512;              // 4 K-atoms x 128 rows
@@ -50,7 +50,7 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr uint32_t kStageTx = 2u * kStageBytes;
 constexpr int kEpiWarps = 8;
 constexpr int kSlotBytes = 32 * 128;            // 32 rows x 128 bytes (one TMA store box)
-constexpr int kSlots = 2;
+constexpr int kSlots = 1;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol0 = 0, kAccCol1 = 192;
@@ -63,7 +63,6 @@ constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
 struct Smem {
   uint8_t stage[kStages][kStageBytes];          // 1024-aligned (kStageBytes % 1024 == 0)
   uint8_t out[kEpiWarps][kSlots][kSlotBytes];
-  float bias[kEpiWarps][BN / 2];
   uint64_t full[kStages], empty[kStages];
   uint64_t acc_full[2], acc_free[2], mma_done;
   uint32_t tmem_base;
@@ -253,7 +252,6 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     const int cols = p.out_f32 ? 32 : 64;          // columns per chunk
     const int nchunks = (BN / 2) / cols;           // chunks per half
     const int overlap_chunks = 64 / cols;          // chunks covering the 64 shared columns
-    float* bias = sm.bias[e];
     int i = 0;
     for (int tile = pair; tile < num_tiles; tile += npairs, ++i) {
       const int tm = tile / p.tiles_n, tn = tile % p.tiles_n;
@@ -263,12 +261,6 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       // buffer 0 shares its top 64 columns (half 1), buffer 1 its bottom 64 (half 0)
       const bool holds_overlap = (b == 0) == (h == 1);
       const uint32_t free_bar = mapa_shared(smem_u32(&sm.acc_free[b]), 0);
-      __syncwarp();
-      for (int c = lane; c < BN / 2; c += 32) {
-        const int n = n0 + c;
-        bias[c] = (p.bias && n < p.N) ? bf16_bits_to_f32(p.bias[n]) : 0.f;
-      }
-      __syncwarp();
       if (!holds_overlap) {
         // this warp is done with the previous tile: release this one for it
         tc_fence_before();
@@ -282,6 +274,16 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         // bottom: the shared columns come first
         const int c = (b == 0 && h == 1) ? nchunks - 1 - step : step;
         uint8_t* buf = sm.out[e][step % kSlots];
+        // this chunk's bias, the same for every lane (issued before the TMEM wait)
+        float bv[64];
+        const int nb = n0 + cols * c;
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          uint32_t w = 0;
+          if (p.bias && k < cols && nb + k < p.N) w = __ldg(reinterpret_cast<const uint32_t*>(p.bias + nb + k));
+          bv[k] = bf16_bits_to_f32(w & 0xFFFFu);
+          bv[k + 1] = bf16_bits_to_f32(w >> 16);
+        }
         uint32_t v[32], v2[32];
         tmem_ld32(tbase + cols * c, v);
         if (!p.out_f32) tmem_ld32(tbase + cols * c + 32, v2);
@@ -296,19 +298,16 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (p.out_f32) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float4 bv = *reinterpret_cast<const float4*>(bias + 32 * c + 4 * u);
-            const float o0 = fmaf(alpha, __uint_as_float(v[4 * u]), bv.x);
-            const float o1 = fmaf(alpha, __uint_as_float(v[4 * u + 1]), bv.y);
-            const float o2 = fmaf(alpha, __uint_as_float(v[4 * u + 2]), bv.z);
-            const float o3 = fmaf(alpha, __uint_as_float(v[4 * u + 3]), bv.w);
+            const float o0 = fmaf(alpha, __uint_as_float(v[4 * u]), bv[4 * u]);
+            const float o1 = fmaf(alpha, __uint_as_float(v[4 * u + 1]), bv[4 * u + 1]);
+            const float o2 = fmaf(alpha, __uint_as_float(v[4 * u + 2]), bv[4 * u + 2]);
+            const float o3 = fmaf(alpha, __uint_as_float(v[4 * u + 3]), bv[4 * u + 3]);
             *reinterpret_cast<float4*>(buf + lane * 128 + ((u ^ (lane & 7)) * 16)) = make_float4(o0, o1, o2, o3);
           }
         } else {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const float4 b0 = *reinterpret_cast<const float4*>(bias + 64 * c + 8 * u);
-            const float4 b1 = *reinterpret_cast<const float4*>(bias + 64 * c + 8 * u + 4);
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const float* bb = bv + 8 * u;
             uint32_t w4[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

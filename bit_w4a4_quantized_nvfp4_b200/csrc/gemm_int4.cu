@@ -7,14 +7,19 @@
 // B200 has no 4-bit integer MMA, so the packed codes are widened to int8 in
 // shared memory and multiplied with tcgen05.mma kind::i8. Each 64-wide group
 // needs its own scale, so every group gets its own int32 accumulator in
-// tensor memory (two buffers, alternating) that the epilogue warps drain into
-// an fp32 running sum held in registers; the int32 group sums are exact.
-// The low-rank term P L2 is one tcgen05.mma kind::f16 per tile into a third
-// TMEM region.
+// tensor memory (three buffers in rotation, so the MMAs run up to two groups
+// ahead of the drain) that the epilogue warps drain into an fp32 running sum
+// held in registers; the int32 group sums are exact. The low-rank term P L2
+// is one tcgen05.mma kind::f16 per tile into a fourth TMEM region.
 //
-// Roles (288 threads): warps 0-3 producers (load packed codes, sign-extend to
-// int8, write the K-major core-matrix layout, arrive on the stage barrier),
-// warp 4 TMEM allocator + single-thread MMA issuer, warps 5-8 epilogue.
+// Roles (416 threads): warps 0-3 producers (load packed codes one group ahead,
+// sign-extend to int8, write the K-major core-matrix layout, arrive on the
+// stage barrier), warp 4 TMEM allocator + MMA issuer, warps 5-12 epilogue, two
+// per TMEM lane quadrant, each holding the running sums of 64 columns.
+// The epilogue turns each exact int32 group sum s (|s| <= 64 * 64) into fp32
+// without the conversion unit: the bits of s + 0x4B400000 are the float
+// 2^23 + 2^22 + s, so one integer add and one float subtraction give s
+// exactly; the scaling then runs as packed f32x2 multiplies and FMAs.
 // Tile 128 x 128, one 64-wide group per pipeline stage, 4 stages.
 // INT4 weight scales are stored group-major [K/64, N] so one group's 128
 // column scales are contiguous.
@@ -30,10 +35,11 @@ constexpr int kOpBytes = 128 * BKG;             // int8 tile, 8 KB
 constexpr int kChunkStride = 128 * 16;          // bytes between 16-byte K chunks
 constexpr int kMaxR = 64;
 constexpr int kLrBytes = 128 * kMaxR * 2;       // 16 KB
-constexpr int kProdWarps = 4, kEpiWarps = 4;
+constexpr int kProdWarps = 4, kEpiWarps = 8;
 constexpr int kThreads = 32 * (kProdWarps + 1 + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kLrCol = 256;
+constexpr int kAccBufs = 3;                     // int32 group accumulators, 128 columns each
+constexpr uint32_t kLrCol = 128 * kAccBufs;     // 384: the low-rank fp32 accumulator
 
 // kind::i8: D s32, A/B signed int8, K-major, M = 128, N = 128
 constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -47,9 +53,9 @@ struct Smem {
   uint8_t b[kStages][kOpBytes];
   uint8_t p[kLrBytes];
   uint8_t l[kLrBytes];
-  float sw[kEpiWarps][BN];
+  float sw[kEpiWarps][BN / 2];
   uint64_t full[kStages], empty[kStages];
-  uint64_t accf[2], acce[2];
+  uint64_t accf[kAccBufs], acce[kAccBufs];
   uint64_t lr_full, lr_empty, lr_accf, lr_acce, mma_done;
   uint32_t tmem_base;
 };
@@ -90,7 +96,7 @@ gemm_int4_kernel(const Params p) {
       mbar_init(&sm.full[s], 32 * kProdWarps);
       mbar_init(&sm.empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&sm.accf[i], 1);
       mbar_init(&sm.acce[i], kEpiWarps);
     }
@@ -131,21 +137,27 @@ gemm_int4_kernel(const Params p) {
         fence_proxy_async_smem();
         mbar_arrive(&sm.lr_full);
       }
-      for (int g = 0; g < p.NG; ++g, ++it) {
-        const int s = it % kStages;
-        if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
-        uint4 ca[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        uint4 cb[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        if (m < p.M) {
+      // this row's packed codes of one group, loaded a group ahead of their use
+      auto load_codes = [&](int g, uint4 (&ca)[2], uint4 (&cb)[2]) {
+        ca[0] = ca[1] = cb[0] = cb[1] = make_uint4(0, 0, 0, 0);
+        if (g < p.NG && m < p.M) {
           const uint4* src = reinterpret_cast<const uint4*>(p.xc + (size_t)m * (p.K / 2) + 32 * g);
           ca[0] = src[0];
           ca[1] = src[1];
         }
-        if (n < p.N) {
+        if (g < p.NG && n < p.N) {
           const uint4* src = reinterpret_cast<const uint4*>(p.wc + (size_t)n * (p.K / 2) + 32 * g);
           cb[0] = src[0];
           cb[1] = src[1];
         }
+      };
+      uint4 na[2], nb2[2];
+      load_codes(0, na, nb2);
+      for (int g = 0; g < p.NG; ++g, ++it) {
+        const int s = it % kStages;
+        const uint4 ca[2] = {na[0], na[1]}, cb[2] = {nb2[0], nb2[1]};
+        load_codes(g + 1, na, nb2);
+        if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint32_t wa[4] = {ca[h].x, ca[h].y, ca[h].z, ca[h].w};
@@ -173,9 +185,9 @@ gemm_int4_kernel(const Params p) {
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tl) {
         for (int g = 0; g < p.NG; ++g, ++it, ++gc) {
           const int s = it % kStages;
-          const int ab = gc & 1;
+          const int ab = gc % kAccBufs;
           if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
-          if (!warp_wait(&sm.acce[ab], ((gc >> 1) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
+          if (!warp_wait(&sm.acce[ab], ((gc / kAccBufs) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a = smem_u32(sm.a[s]), b = smem_u32(sm.b[s]);
           uint64_t da[2], db[2];
@@ -217,37 +229,49 @@ gemm_int4_kernel(const Params p) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - (kProdWarps + 1);   // 0..3
+    const int ew = warp - (kProdWarps + 1);   // 0..7
     const int q = warp & 3;                    // TMEM lane quadrant
+    const int h = ew >> 2;                     // columns [64 h, 64 h + 64)
     float* sw = sm.sw[ew];
     uint32_t gc = 0, tl = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
-      const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN;
+      const int m0 = (tile / p.tiles_n) * BM, n0 = (tile % p.tiles_n) * BN + 64 * h;
       const int m = m0 + 32 * q + lane;
-      float acc[BN];
+      float acc[64];
 #pragma unroll
-      for (int j = 0; j < BN; ++j) acc[j] = 0.f;
+      for (int j = 0; j < 64; ++j) acc[j] = 0.f;
       bool ok = true;
-      for (int g = 0; g < p.NG; ++g, ++gc) {
-        const int ab = gc & 1;
-        // this group's column scales (group-major layout: contiguous in n)
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < BN / 32; ++i) {
-          const int n = n0 + lane + 32 * i;
-          sw[lane + 32 * i] = n < p.N ? bf16_bits_to_f32(p.ws[(size_t)g * p.N + n]) : 0.f;
+      // this lane's two column scales and its row scale of a group (loaded a group ahead)
+      auto load_scales = [&](int g, uint32_t& w2, float& sx) {
+        w2 = 0;
+        sx = 0.f;
+        if (g < p.NG) {
+          const int n = n0 + 2 * lane;
+          if (n < p.N) w2 = *reinterpret_cast<const uint32_t*>(p.ws + (size_t)g * p.N + n);
+          if (m < p.M) sx = bf16_bits_to_f32(p.xs[(size_t)m * p.NG + g]);
         }
-        const float sx = m < p.M ? bf16_bits_to_f32(p.xs[(size_t)m * p.NG + g]) : 0.f;
+      };
+      uint32_t nw2;
+      float nsx;
+      load_scales(0, nw2, nsx);
+      for (int g = 0; g < p.NG; ++g, ++gc) {
+        const int ab = gc % kAccBufs;
+        const uint32_t w2 = nw2;
+        const float sx = nsx;
+        load_scales(g + 1, nw2, nsx);
+        // this group's 64 column scales, shared by the warp's lanes
         __syncwarp();
-        if (!mbar_wait(&sm.accf[ab], (gc >> 1) & 1, p.wait_ns, p.err)) { ok = false; break; }
+        *reinterpret_cast<float2*>(sw + 2 * lane) = make_float2(bf16_bits_to_f32(w2 & 0xFFFFu), bf16_bits_to_f32(w2 >> 16));
+        __syncwarp();
+        if (!mbar_wait(&sm.accf[ab], (gc / kAccBufs) & 1, p.wait_ns, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tb = tmem + 128 * ab + ((uint32_t)(32 * q) << 16);
+        const uint32_t tb = tmem + 128 * ab + 64 * h + ((uint32_t)(32 * q) << 16);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tmem_ld32(tb + 32 * c, v);
           tmem_ld_wait();
-          if (c == BN / 32 - 1) {
+          if (c == 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.acce[ab]);
@@ -261,8 +285,24 @@ gemm_int4_kernel(const Params p) {
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              acc[32 * c + j] = fmaf(__fmul_rn(sx, sw[32 * c + j]), (float)(int32_t)v[j], acc[32 * c + j]);
+            for (int j = 0; j < 32; j += 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(sw + 32 * c + j);
+              // exact int32 -> fp32 through the bits of 2^23 + 2^22 + s
+              const float2 f01 = __fadd2_rn(make_float2(__uint_as_float(v[j] + 0x4B400000u),
+                                                        __uint_as_float(v[j + 1] + 0x4B400000u)),
+                                            make_float2(-12582912.0f, -12582912.0f));
+              const float2 f23 = __fadd2_rn(make_float2(__uint_as_float(v[j + 2] + 0x4B400000u),
+                                                        __uint_as_float(v[j + 3] + 0x4B400000u)),
+                                            make_float2(-12582912.0f, -12582912.0f));
+              const float2 s01 = __fmul2_rn(make_float2(s4.x, s4.y), make_float2(sx, sx));
+              const float2 s23 = __fmul2_rn(make_float2(s4.z, s4.w), make_float2(sx, sx));
+              const float2 a01 = __ffma2_rn(s01, f01, make_float2(acc[32 * c + j], acc[32 * c + j + 1]));
+              const float2 a23 = __ffma2_rn(s23, f23, make_float2(acc[32 * c + j + 2], acc[32 * c + j + 3]));
+              acc[32 * c + j] = a01.x;
+              acc[32 * c + j + 1] = a01.y;
+              acc[32 * c + j + 2] = a23.x;
+              acc[32 * c + j + 3] = a23.y;
+            }
           }
         }
       }
@@ -270,9 +310,9 @@ gemm_int4_kernel(const Params p) {
       if (has_lr) {
         if (!mbar_wait(&sm.lr_accf, tl & 1, p.wait_ns, p.err)) break;
         tc_fence_after();
-        const uint32_t tb = tmem + kLrCol + ((uint32_t)(32 * q) << 16);
+        const uint32_t tb = tmem + kLrCol + 64 * h + ((uint32_t)(32 * q) << 16);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tmem_ld32(tb + 32 * c, v);
           tmem_ld_wait();
@@ -284,9 +324,9 @@ gemm_int4_kernel(const Params p) {
         if (lane == 0) mbar_arrive(&sm.lr_acce);
       }
       if (p.out == 2 || m >= p.M) continue;
-      // y = acc + bias; each thread writes its row's 128 columns
+      // y = acc + bias; each thread writes its row's 64 columns
 #pragma unroll
-      for (int c = 0; c < BN / 8; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const int nb = n0 + 8 * c;
         if (nb >= p.N) break;  // N % 8 == 0: a group of 8 columns is all in or all out
         float o[8];

@@ -52,6 +52,7 @@ WORKLOAD = "c3_qkv_nvfp4"
 METRIC = "SVDQ W4A4-NVFP4 linear TFLOPS, % dense FP4 peak (M4608 K3072 N9216 r32)"
 FP4_DENSE_SPEC_TFLOPS = 9000.0
 NOMINAL_FP4_OVER_BF16 = 4.0     # 9 PF / 2.25 PF dense
+NOMINAL_INT8_OVER_BF16 = 2.0    # 4.5 POPS / 2.25 PF dense
 L2_FLUSH_BYTES = 512 << 20
 GEMM_SOURCE = os.path.join(ROOT, "bit_w4a4_quantized_nvfp4_b200", "csrc", "gemm_nvfp4.cu")
 # {sha256 of the GEMM kernel source: DRAM bytes per launch from an ncu capture of the workload}
@@ -309,12 +310,50 @@ def run_cuda(args):
         out["cpu_baseline"] = cpu_baseline(d, rows=args.cpu_rows)
     if rank == 0 and not args.no_awq:
         out["awq_gemv"] = bench_awq(svdq, P)
+    if rank == 0 and not args.no_int4:
+        out["int4_linear"] = bench_int4(svdq, P)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
         import torch.distributed as dist
 
         dist.destroy_process_group()
+
+
+def bench_int4(svdq, P, steps=10):
+    """The INT4 variant of the layer (M4608 K3072 N9216 r32, symmetric INT4
+    g64 activations and weights): one step = svdq_quantize_act + svdq_w4a4_linear,
+    L2 flushed before each step, against the dense INT8 tensor peak (the int4
+    codes are widened to int8 for the MMA)."""
+    name = "c5_qkv_int4"
+    c = synth.CONFIGS[name]
+    M, K, N, r = c["M"], c["K"], c["N"], c["r"]
+    d = synth.config_layer(name)
+    L1, L2, b = bf16_dev(d["L1"]), bf16_dev(d["L2"]), bf16_dev(d["b"])
+    x = bf16_dev(d["x"])
+    pw = svdq.pack_weight("int4", torch.from_numpy(d["W"]).cuda(), torch.from_numpy(d["lam"]).cuda(), L1, L2)
+    qa = svdq.quantize_act(x, pw, L1)
+    y = svdq.w4a4_linear(qa, pw, b)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ms = []
+    for i in range(steps + 2):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        svdq.quantize_act(x, pw, L1, out=qa)
+        svdq.w4a4_linear(qa, pw, b, out=y)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            ms.append(e0.elapsed_time(e1))
+    svdq.device_error()
+    t = statistics.mean(ms)
+    tops = 2.0 * M * N * K / (t * 1e-3) / 1e12
+    peak = P["bf16"] * NOMINAL_INT8_OVER_BF16
+    return {"workload": f"svdq_w4a4 int4 g64 M{M} K{K} N{N} r{r}", "ms_per_step": round(t, 4),
+            "value": round(tops, 1), "unit": "TOPS", "peak": round(peak, 1),
+            "peak_source": f"{P['source']} bf16 burst {P['bf16']} x nominal int8/bf16 ratio 2",
+            "frac": round(tops / peak, 4), "steps": steps}
 
 
 def bench_awq(svdq, P):
@@ -425,6 +464,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-awq", action="store_true")
+    ap.add_argument("--no-int4", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

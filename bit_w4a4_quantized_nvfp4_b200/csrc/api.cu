@@ -131,7 +131,7 @@ const char* svdq_status_str(svdq_status s) {
 size_t svdq_scale_bytes(svdq_precision p, int rows, int K) {
   if (rows < 0 || K <= 0 || K % 64) return 0;
   if (p == SVDQ_NVFP4) return (size_t)((rows + 127) / 128) * 128 * (size_t)(K / 16);
-  if (p == SVDQ_INT4) return (size_t)rows * (size_t)(K / 64) * 2;
+  if (p == SVDQ_INT4) return (size_t)rows * (size_t)int4_act_scale_pitch(K) * 2;
   return 0;
 }
 

@@ -272,6 +272,11 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
     } else {
       for (int j = 0; j < gn; ++j) group(j);
     }
+    // release the stage only once its weights have gone through the MMAs
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) consumed(tot[mt][i]);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }

@@ -117,6 +117,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// Releasing a shared-memory stage right after issuing loads from it is not
+// safe: the arrive can complete before the loads have read the stage, and the
+// next (async-proxy) write then overtakes them. A consumer therefore releases
+// a stage only after instructions that use the loaded values; `consumed(v)`
+// keeps the computation of v (and so the loads it depends on) ahead of the
+// next volatile instruction, e.g. the release itself.
+__device__ __forceinline__ void consumed(float v) { asm volatile("" ::"f"(v)); }
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -280,6 +288,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// The registers written by tcgen05.ld hold their values only once
+// tcgen05.wait::ld has returned, but the compiler sees them as defined by the
+// load itself and may move arithmetic on them above the wait. Passing each
+// through an empty volatile asm after the wait pins every use below it.
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
 
 // --------------------------------------------------------------------------
 // shared-memory matrix descriptors (tcgen05)

@@ -56,6 +56,11 @@ struct AwqArgs {
 };
 cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 
+// Row pitch, in scales, of the INT4 activation scales [M, K/64]: padded to a
+// multiple of 8 so that every row starts on a 16-byte boundary (the GEMM
+// reads them with TMA).
+__host__ __device__ inline int int4_act_scale_pitch(int K) { return ((K / 64 + 7) / 8) * 8; }
+
 struct GemmArgs {
   const uint8_t* x_codes;
   const void* x_scales;

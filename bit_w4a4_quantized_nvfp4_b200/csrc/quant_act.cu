@@ -122,7 +122,8 @@ struct Cfg {
 };
 
 // PREC 0 = NVFP4 (group 16, E4M3 scales in the tiled layout), 1 = INT4
-// (group 64, bf16 scales row-major). NT = r / 8 tiles of the P output.
+// (group 64, bf16 scales row-major, row pitch int4_act_scale_pitch). NT = r / 8
+// tiles of the P output.
 template <int PREC, int NT>
 __global__ void __launch_bounds__(kThreadsQA, 1)
 quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
@@ -207,7 +208,7 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   uint8_t* scale_ptr =
       PREC == 0 ? static_cast<uint8_t*>(a.scales) + ((size_t)(m_c / 128) * (K / 64) + kp) * 512 + 16 * (m_c % 32) +
                       4 * ((m_c % 128) / 32)
-                : static_cast<uint8_t*>(a.scales) + ((size_t)m_c * (K / 64) + kp) * 2;
+                : static_cast<uint8_t*>(a.scales) + ((size_t)m_c * int4_act_scale_pitch(K) + kp) * 2;
 
   float acc[NT > 0 ? NT : 1][4];
 #pragma unroll
@@ -326,7 +327,14 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       }
     }
     // the stage may be refilled (by the async proxy) once every lane is past
-    // its reads and writes of it
+    // its reads and writes of it: the P MMAs (which use the last reads of the
+    // stage) are kept ahead of the release
+    if constexpr (NT > 0) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) consumed(acc[t][i]);
+    }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);

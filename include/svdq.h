@@ -74,9 +74,11 @@ const char* svdq_status_str(svdq_status s);
  *   rb*128 + 32*i + j (i < 4, j < 32) for K block 4*ka + c (c < 4) is at byte
  *   16*j + 4*i + c. rows are padded up to a multiple of 128 (padding scales 0).
  *   Size = ceil(rows/128) * 128 * K/16.
- * INT4: bf16, one per (row, 64-block): activations row-major [M, K/64]; weights
- *   group-major [K/64, N] (one group's column scales contiguous for the GEMM
- *   epilogue). Size = rows * K/64 * 2.
+ * INT4: bf16, one per (row, 64-block): activations row-major [M, K/64] with
+ *   the row pitch padded to pitch = 8 * ceil(K/512) scales (every row starts on
+ *   a 16-byte boundary; the padding is never read); weights group-major
+ *   [K/64, N] (one group's column scales contiguous for the GEMM epilogue).
+ *   Size = rows * pitch * 2 (also enough for the weights' K/64 * N * 2).
  * Returns 0 for invalid arguments. */
 size_t svdq_scale_bytes(svdq_precision p, int rows, int K);
 

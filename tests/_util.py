@@ -16,6 +16,19 @@ def untile_nvfp4_scales(tiled: np.ndarray, rows: int, K: int) -> np.ndarray:
     return tiled[idx]
 
 
+def int4_act_scale_pitch(K: int) -> int:
+    """Row pitch (in scales) of INT4 activation scales: K/64 rounded up to a
+    multiple of 8, so that every row starts on a 16-byte boundary."""
+    return ((K // 64 + 7) // 8) * 8
+
+
+def unpad_int4_act_scales(raw: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """INT4 activation scale bytes (row pitch int4_act_scale_pitch) -> plain
+    bf16 bits [rows, K/64]."""
+    pitch = int4_act_scale_pitch(K)
+    return np.asarray(raw, np.uint8).reshape(-1)[: rows * pitch * 2].view(np.uint16).reshape(rows, pitch)[:, : K // 64]
+
+
 def bf16_ulp(v: np.ndarray) -> np.ndarray:
     a = np.abs(np.asarray(v, np.float64))
     e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))

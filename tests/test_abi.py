@@ -50,6 +50,8 @@ def test_scale_sizes(lib):
     assert lib.svdq_scale_bytes(0, 256, 1024) == 256 * 64
     assert lib.svdq_scale_bytes(0, 200, 1024) == 256 * 64   # rows padded to 128
     assert lib.svdq_scale_bytes(1, 200, 1024) == 200 * 16 * 2
+    assert lib.svdq_scale_bytes(1, 200, 192) == 200 * 8 * 2  # INT4 row pitch: 3 groups padded to 8
+    assert lib.svdq_scale_bytes(1, 7, 3072) == 7 * 48 * 2
     assert lib.svdq_scale_bytes(0, 8, 100) == 0             # K % 64 != 0
     assert lib.svdq_lr_up_elems(0, 9216, 32) == 9216 * 64
     assert lib.svdq_lr_up_elems(1, 9216, 32) == 9216 * 32

@@ -14,7 +14,8 @@ import torch
 import oracle
 import synth
 import bit_w4a4_quantized_nvfp4_b200 as svdq
-from tests._util import bf16_ulp, check_bf16_output, check_f32_output, untile_nvfp4_scales
+from tests._util import (bf16_ulp, check_bf16_output, check_f32_output, int4_act_scale_pitch,
+                         unpad_int4_act_scales, untile_nvfp4_scales)
 
 pytestmark = pytest.mark.gpu
 
@@ -84,6 +85,8 @@ def compare_pack_and_act(prec, d, pw, qa, w, a):
     if prec == "nvfp4":
         assert np.array_equal(untile_nvfp4_scales(pw.scales.cpu().numpy(), N, K), w["scales"])
         assert np.array_equal(untile_nvfp4_scales(qa.scales.cpu().numpy(), M, K), a["scales"])
+    else:
+        assert np.array_equal(unpad_int4_act_scales(qa.scales.cpu().numpy(), M, K), a["scales"])
     assert np.array_equal(qa.codes.cpu().numpy(), a["codes"])
     if r:
         # P = bf16(x_hat L1): the kernel accumulates in fp32 on tensor cores, the
@@ -188,8 +191,7 @@ def test_int4_pack_and_quantize_match_oracle(M, K, N, r):
     w = oracle.pack_weight("int4", d["W"], d["lam"], d["L1"], d["L2"])
     a = oracle.quantize_act("int4", d["x"], w["inv_lam"], 1.0, d["L1"])
     compare_pack_and_act("int4", d, pw, qa, w, a)
-    assert np.array_equal(qa.scales.cpu().numpy()[: M * (K // 64) * 2].view(np.uint16).reshape(M, K // 64),
-                          a["scales"])
+    assert np.array_equal(unpad_int4_act_scales(qa.scales.cpu().numpy(), M, K), a["scales"])
     # weight scales are stored group-major [K/64, N]
     assert np.array_equal(pw.scales.cpu().numpy()[: N * (K // 64) * 2].view(np.uint16).reshape(K // 64, N).T,
                           w["scales"])
@@ -252,7 +254,7 @@ def test_c5_int4_full_size():
     compare_pack_and_act("int4", d, pw, qa, w, a)
     check_bf16_output(as_f32(bf16_np(y))[rows], yo, as_f32(oracle.bf16_rn(yo)))
     sub = svdq.QuantAct(qa.prec, 48, qa.K, qa.r, qa.codes[:48].contiguous(),
-                        qa.scales[: 48 * (qa.K // 64) * 2].contiguous(),
+                        qa.scales[: 48 * int4_act_scale_pitch(qa.K) * 2].contiguous(),
                         qa.P[:48].contiguous() if qa.P is not None else None)
     gs = svdq.w4a4_linear(sub, pw, None, out_dtype="i32_groups")
     torch.cuda.synchronize()

@@ -107,6 +107,9 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
   int* abort_flag = reinterpret_cast<int*>(xbar + 2);
   float* red = reinterpret_cast<float*>(abort_flag + 4);  // phases 1.. partial sums [kh-1][rt][mt][lane][4]
 
+  // the next kernel in the stream may be scheduled as SMs free up; it waits
+  // for this one before it reads anything this one writes
+  if (threadIdx.x == 0) launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesA; ++s) {
       mbar_init(&full[s], 1);
@@ -129,15 +132,20 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
     };
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
-      // activations (one bulk copy per row) and this CTA's rows of scales and
-      // zero points (contiguous: rows n0 .. n0 + rows - 1, 16-byte aligned)
+      // this CTA's rows of scales and zero points (contiguous: rows n0 ..
+      // n0 + rows - 1, 16-byte aligned) and the first weight stages: packed
+      // weights are never written by an earlier kernel, so they stream
+      // before the wait for the previous kernel in the stream
       const uint32_t sz_bytes = (uint32_t)(min(kRowsA, N - n0) * L.sz_pitch);
       mbar_expect_tx(xbar, (uint32_t)(M * 2 * K) + 2 * sz_bytes);
-      for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
       bulk_load(base + L.off_s, a.s + (size_t)n0 * ng, sz_bytes, xbar);
       bulk_load(base + L.off_z, a.z + (size_t)n0 * ng, sz_bytes, xbar);
       // the first stages need no release
       for (; c < nst && c < kStagesA; ++c) issue_stage(c);
+      // the activations may come from the previous kernel (one bulk copy per
+      // row); y is written only after they have arrived
+      grid_dependency_wait();
+      for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
       for (; c < nst; ++c) {
         const int s = c % kStagesA;
         if (!mbar_wait(&empty[s], ((c / kStagesA) - 1) & 1, wait_ns, err)) {
@@ -343,7 +351,20 @@ cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_
     const size_t smem = (size_t)AwqLayout(b.M, a.K).total + 1024;
     cudaError_t e = cudaFuncSetAttribute(awq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    awq_kernel<<<grid, kThreadsA, smem, s>>>(tm_q, b, err, wait_ns);
+    // programmatic dependent launch: this grid may start while the previous
+    // kernel in the stream finishes (see the kernel's wait before x)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreadsA);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, awq_kernel, tm_q, b, err, wait_ns);
+    if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

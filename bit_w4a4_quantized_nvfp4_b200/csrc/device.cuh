@@ -22,6 +22,13 @@ __device__ __forceinline__ void raise_error(unsigned* err, unsigned bit) {
   if (err) atomicOr(err, bit);
 }
 
+// Programmatic dependent launch. `grid_dependency_wait` returns once every
+// kernel this grid depends on (the previous one in the stream) has completed
+// and its memory operations are visible; `launch_dependents` lets the next
+// kernel in the stream be scheduled before this one completes.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -69,6 +69,7 @@ def lib():
             "orc_int4_group_sums": (i32, [i32, i32, i32, P, P, P]),
             "orc_awq_pack_weight": (i32, [i32, i32, P, P, P, P]),
             "orc_awq_linear": (i32, [i32, i32, i32, P, P, P, P, P, P]),
+            "orc_qkv_norm_rope": (i32, [i32, i32, i32, P, P, P, C.c_double, P, P, P]),
             "orc_bf16_rn_f64_array": (None, [P, i64, P]),
             "orc_e4m3_rn_array": (None, [P, i64, P]),
             "orc_e2m1_rn_array": (None, [P, i64, P]),
@@ -247,6 +248,24 @@ def int4_group_sums(x_codes, w_codes):
     rc = lib().orc_int4_group_sums(M, K, N, _p(x_codes), _p(w_codes), _p(out))
     if rc:
         raise ValueError(f"orc_int4_group_sums: {rc}")
+    return out
+
+
+def qkv_norm_rope(y, heads: int, head_dim: int, wq, wk, eps: float, cos, sin):
+    """Fused QKV epilogue on the unrounded layer output y [M, 3*heads*head_dim]
+    (Q, K, V in that order): per-head RMSNorm of Q and K with bf16 weights wq,
+    wk [head_dim], then the rotary embedding of adjacent pairs with cos, sin
+    [M, head_dim/2]; V passes through. Returns float64, unrounded."""
+    y = _c(y, np.float64)
+    M = y.shape[0]
+    assert y.shape[1] == 3 * heads * head_dim
+    cos = _c(cos, np.float32).reshape(M, head_dim // 2)
+    sin = _c(sin, np.float32).reshape(M, head_dim // 2)
+    out = np.zeros_like(y)
+    rc = lib().orc_qkv_norm_rope(M, heads, head_dim, _p(y), _p(_c(wq, np.uint16)), _p(_c(wk, np.uint16)),
+                                 float(eps), _p(cos), _p(sin), _p(out))
+    if rc:
+        raise ValueError(f"orc_qkv_norm_rope: {rc}")
     return out
 
 

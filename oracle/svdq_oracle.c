@@ -532,6 +532,50 @@ int orc_awq_linear(int M, int K, int N, const uint16_t* x, const uint8_t* q, con
 }
 
 /* ------------------------------------------------------------------------- */
+/* fused QKV epilogue: per-head RMSNorm of Q and K, then rotary embedding     */
+/* ------------------------------------------------------------------------- */
+/* The grouped projection's output y [M, 3*H*D] holds Q, K and V concatenated
+ * along the output dimension in that order, each as H heads of D columns
+ * (Diffusers "Nunchaku Lite" page, section on fused kernels: Q/K/V projection
+ * combined with RMSNorm and RoPE; the grouped to_qkv module). For every row m
+ * and every head of Q (weight wq) and of K (weight wk):
+ *   u[d]      = v[d] / sqrt(mean_d(v^2) + eps) * w[d]          (RMSNorm over D)
+ *   out[2i]   = u[2i] cos[m,i] - u[2i+1] sin[m,i]               (rotary embedding,
+ *   out[2i+1] = u[2i] sin[m,i] + u[2i+1] cos[m,i]                pairs (2i, 2i+1))
+ * V is passed through. y is the unrounded layer output (the fusion reads the
+ * GEMM accumulator); everything is in double and the caller rounds once.
+ * wq, wk: bf16 [D]; cos, sin: fp32 [M, D/2]; out: [M, 3*H*D]. */
+int orc_qkv_norm_rope(int M, int H, int D, const double* y, const uint16_t* wq, const uint16_t* wk,
+                      double eps, const float* cos_t, const float* sin_t, double* out) {
+  if (M < 0 || H <= 0 || D <= 0 || D % 2 || eps < 0.0) return ORC_EINVAL;
+  const size_t N = (size_t)3 * H * D;
+#pragma omp parallel for schedule(static)
+  for (int m = 0; m < M; ++m) {
+    const double* yr = y + (size_t)m * N;
+    double* orow = out + (size_t)m * N;
+    for (size_t n = 2 * (size_t)H * D; n < N; ++n) orow[n] = yr[n];  /* V */
+    double* u = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int sec = 0; sec < 2; ++sec) {
+      const uint16_t* w = sec == 0 ? wq : wk;
+      for (int h = 0; h < H; ++h) {
+        const size_t off = ((size_t)sec * H + h) * D;
+        double ss = 0.0;
+        for (int d = 0; d < D; ++d) ss += yr[off + d] * yr[off + d];
+        const double inv = 1.0 / sqrt(ss / D + eps);
+        for (int d = 0; d < D; ++d) u[d] = yr[off + d] * inv * (double)orc_bf16_to_f32(w[d]);
+        for (int i = 0; i < D / 2; ++i) {
+          const double c = (double)cos_t[(size_t)m * (D / 2) + i], sn = (double)sin_t[(size_t)m * (D / 2) + i];
+          orow[off + 2 * i] = u[2 * i] * c - u[2 * i + 1] * sn;
+          orow[off + 2 * i + 1] = u[2 * i] * sn + u[2 * i + 1] * c;
+        }
+      }
+    }
+    free(u);
+  }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------- */
 /* array forms of the format conversions (for the tests)                     */
 /* ------------------------------------------------------------------------- */
 

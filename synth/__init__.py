@@ -11,6 +11,7 @@ from .inputs import (  # noqa: F401
     CONFIGS,
     config_layer,
     awq_inputs,
+    qkv_epilogue_inputs,
     bf16_bits,
     bf16_bits_to_f32,
     normal,

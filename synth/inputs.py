@@ -41,6 +41,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 # tensor ids inside one seed
 _T_X, _T_W, _T_B, _T_XOUT, _T_WOUT, _T_OMEGA = 1, 2, 3, 4, 5, 6
+_T_WQ, _T_WK = 7, 8  # RMSNorm weights of the fused QKV epilogue
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -180,6 +181,21 @@ def awq_inputs(seed: int, M: int, K: int, N: int, w_std=0.02):
     x = bf16_bits(normal(seed, _T_X, M * K).reshape(M, K))
     W = (normal(seed, _T_W, K * N).reshape(K, N) * w_std).astype(np.float32)
     return dict(x=x, W=W, M=M, K=K, N=N)
+
+
+def qkv_epilogue_inputs(seed: int, M: int, head_dim: int, heads: int, rope_base: float = 10000.0):
+    """Inputs of the fused QKV epilogue on a grouped Q/K/V projection of `heads`
+    heads of `head_dim` columns per section: RMSNorm weights wq, wk (bf16 bits
+    [head_dim], ~ U(0.5, 1.5), standing in for trained ones) and rotary tables
+    cos, sin (fp32 [M, head_dim/2]) for token positions 0..M-1 with the usual
+    frequencies base^(-2i/head_dim). eps = 1e-6."""
+    wq = bf16_bits(0.5 + uniform(seed, _T_WQ, head_dim))
+    wk = bf16_bits(0.5 + uniform(seed, _T_WK, head_dim))
+    pos = np.arange(M, dtype=np.float64)[:, None]
+    freq = rope_base ** (-2.0 * np.arange(head_dim // 2, dtype=np.float64) / head_dim)[None, :]
+    ang = pos * freq
+    return dict(wq=wq, wk=wk, cos=np.cos(ang).astype(np.float32), sin=np.sin(ang).astype(np.float32),
+                eps=1e-6, heads=heads, head_dim=head_dim)
 
 
 # The five workloads. Sizes, distributions and outlier structure follow the

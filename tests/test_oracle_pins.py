@@ -500,3 +500,121 @@ def test_awq_linear_exact_on_tiny_problem():
             exact = sum(Fraction(float(x[m, k])) * (int(q[n, k]) - Fraction(float(z[n, k // 64])))
                         * Fraction(float(s[n, k // 64])) for k in range(128)) + Fraction(float(bf[n]))
             assert abs(Fraction(y[m, n]) - exact) <= abs(exact) * Fraction(1, 2**48) + Fraction(1, 2**70)
+
+
+# ------------------------------------------------------------------ fused QKV epilogue (RMSNorm + rotary)
+# Pins of oracle.qkv_norm_rope: invariants of a norm followed by a rotation,
+# and relations between oracle calls with different rotation tables; none
+# re-derives the oracle's arithmetic.
+H_Q, D_Q, M_Q = 3, 8, 5
+
+
+def _qkv_case(seed):
+    rng = np.random.default_rng(seed)
+    y = rng.standard_normal((M_Q, 3 * H_Q * D_Q)) * np.exp(rng.uniform(-3, 3, (M_Q, 1)))
+    wq = oracle.bf16_rn(rng.uniform(0.5, 1.5, D_Q))
+    wk = oracle.bf16_rn(rng.uniform(0.5, 1.5, D_Q))
+    theta = rng.uniform(-np.pi, np.pi, (M_Q, D_Q // 2))
+    return y, wq, wk, theta
+
+
+def _rot(theta, sign=1.0):
+    return np.cos(theta).astype(np.float32), (sign * np.sin(theta)).astype(np.float32)
+
+
+def _heads(a, sec):
+    """Section sec (0 Q, 1 K, 2 V) of a [M, 3 H D] array as [M, H, D]."""
+    return a[:, sec * H_Q * D_Q:(sec + 1) * H_Q * D_Q].reshape(a.shape[0], H_Q, D_Q)
+
+
+ONES = oracle.bf16_rn(np.ones(D_Q))
+ZEROS_T = np.zeros((M_Q, D_Q // 2))
+
+
+def test_qkv_unit_weights_no_eps_give_unit_rms_heads():
+    # with w = 1, eps = 0 and no rotation every Q/K head comes out with RMS 1
+    # and points the same way as its input; V is passed through bit for bit
+    y, _, _, _ = _qkv_case(1)
+    c, s = _rot(ZEROS_T)
+    o = oracle.qkv_norm_rope(y, H_Q, D_Q, ONES, ONES, 0.0, c, s)
+    for sec in (0, 1):
+        oh, yh = _heads(o, sec), _heads(y, sec)
+        assert np.allclose(np.sqrt(np.mean(oh ** 2, axis=2)), 1.0, rtol=1e-13)
+        ratio = oh / yh
+        assert np.allclose(ratio, ratio[:, :, :1], rtol=1e-12) and (ratio > 0).all()
+    assert np.array_equal(_heads(o, 2), _heads(y, 2))
+
+
+def test_qkv_quarter_turn_maps_pairs():
+    # a rotation by +90 degrees sends the pair (a, b) to (-b, a)
+    y, wq, wk, _ = _qkv_case(2)
+    c0, s0 = _rot(ZEROS_T)
+    u = oracle.qkv_norm_rope(y, H_Q, D_Q, wq, wk, 1e-6, c0, s0)
+    c, s = np.zeros_like(c0), np.ones_like(s0)
+    o = oracle.qkv_norm_rope(y, H_Q, D_Q, wq, wk, 1e-6, c, s)
+    for sec in (0, 1):
+        uh, oh = _heads(u, sec), _heads(o, sec)
+        assert np.allclose(oh[:, :, 0::2], -uh[:, :, 1::2], rtol=1e-14, atol=0)
+        assert np.allclose(oh[:, :, 1::2], uh[:, :, 0::2], rtol=1e-14, atol=0)
+
+
+def test_qkv_rotation_preserves_pair_norms_and_undoes():
+    # each (2i, 2i+1) pair keeps its length; rotating the (unit-RMS) result by
+    # the opposite angles with w = 1, eps = 0 gives back the unrotated heads
+    y, _, _, theta = _qkv_case(3)
+    c0, s0 = _rot(ZEROS_T)
+    u = oracle.qkv_norm_rope(y, H_Q, D_Q, ONES, ONES, 0.0, c0, s0)
+    c, s = _rot(theta)
+    o = oracle.qkv_norm_rope(y, H_Q, D_Q, ONES, ONES, 0.0, c, s)
+    for sec in (0, 1):
+        uh, oh = _heads(u, sec), _heads(o, sec)
+        nu = np.hypot(uh[:, :, 0::2], uh[:, :, 1::2])
+        no = np.hypot(oh[:, :, 0::2], oh[:, :, 1::2])
+        # cos and sin are given in fp32: cos^2 + sin^2 = 1 to within a few ulp
+        assert np.allclose(no, nu, rtol=1e-6)
+    cb, sb = _rot(theta, -1.0)
+    back = oracle.qkv_norm_rope(o, H_Q, D_Q, ONES, ONES, 0.0, cb, sb)
+    for sec in (0, 1):
+        assert np.allclose(_heads(back, sec), _heads(u, sec), rtol=0, atol=1e-6)
+
+
+def test_qkv_norm_scale_invariant_without_eps():
+    y, wq, wk, theta = _qkv_case(4)
+    c, s = _rot(theta)
+    o1 = oracle.qkv_norm_rope(y, H_Q, D_Q, wq, wk, 0.0, c, s)
+    o2 = oracle.qkv_norm_rope(7.5 * y, H_Q, D_Q, wq, wk, 0.0, c, s)
+    for sec in (0, 1):
+        assert np.allclose(_heads(o2, sec), _heads(o1, sec), rtol=1e-13, atol=1e-15)
+    assert np.array_equal(_heads(o2, 2), 7.5 * _heads(y, 2))
+
+
+def test_qkv_constant_head_closed_form():
+    # a head whose D entries all equal c has mean square c^2, so its output
+    # (no rotation) is c / sqrt(c^2 + eps) * w: eps sits under the root, next to
+    # the mean, not the sum
+    cval, eps = 1e-3, 1e-6
+    y = np.zeros((1, 3 * H_Q * D_Q))
+    y[0, :D_Q] = cval
+    wq = oracle.bf16_rn(np.linspace(0.5, 2.0, D_Q))
+    c, s = _rot(np.zeros((1, D_Q // 2)))
+    o = oracle.qkv_norm_rope(y, H_Q, D_Q, wq, ONES, eps, c, s)
+    expect = cval / np.sqrt(cval ** 2 + eps) * oracle.bf16_to_f32(wq).astype(np.float64)
+    assert np.allclose(o[0, :D_Q], expect, rtol=1e-14)
+    # an all-zero head stays zero
+    assert not o[0, D_Q:2 * H_Q * D_Q].any()
+
+
+def test_qkv_heads_and_sections_are_independent():
+    # changing one head of Q changes only that head; K uses wk and Q uses wq
+    y, wq, wk, theta = _qkv_case(5)
+    c, s = _rot(theta)
+    o = oracle.qkv_norm_rope(y, H_Q, D_Q, wq, wk, 1e-6, c, s)
+    y2 = y.copy()
+    y2[:, 1 * D_Q:2 * D_Q] *= -3.0  # Q head 1
+    o2 = oracle.qkv_norm_rope(y2, H_Q, D_Q, wq, wk, 1e-6, c, s)
+    changed = np.abs(o2 - o).max(axis=0) > 0
+    assert changed[D_Q:2 * D_Q].all() and not changed[:D_Q].any() and not changed[2 * D_Q:].any()
+    o3 = oracle.qkv_norm_rope(y, H_Q, D_Q, wq, ONES, 1e-6, c, s)
+    assert np.array_equal(_heads(o3, 0), _heads(o, 0)) and not np.array_equal(_heads(o3, 1), _heads(o, 1))
+    o4 = oracle.qkv_norm_rope(y, H_Q, D_Q, ONES, wk, 1e-6, c, s)
+    assert np.array_equal(_heads(o4, 1), _heads(o, 1)) and not np.array_equal(_heads(o4, 0), _heads(o, 0))

@@ -43,7 +43,7 @@ def _rank_main(rank, world, port, step_ms, out):
 @pytest.mark.parametrize("step_ms", [(0.125, 0.25), (0.5, 0.0625)])
 def test_step_time_is_the_slowest_rank(step_ms):
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.start_processes(_rank_main, args=(world, _free_port(), step_ms, out), nprocs=world, join=True,
                        start_method="spawn")
     assert out[0] == out[1] == max(step_ms)

@@ -70,6 +70,7 @@ def lib():
             "orc_awq_pack_weight": (i32, [i32, i32, P, P, P, P]),
             "orc_awq_linear": (i32, [i32, i32, i32, P, P, P, P, P, P]),
             "orc_qkv_norm_rope": (i32, [i32, i32, i32, P, P, P, C.c_double, P, P, P]),
+            "orc_gelu_bf16": (None, [P, i64, P]),
             "orc_bf16_rn_f64_array": (None, [P, i64, P]),
             "orc_e4m3_rn_array": (None, [P, i64, P]),
             "orc_e2m1_rn_array": (None, [P, i64, P]),
@@ -267,6 +268,20 @@ def qkv_norm_rope(y, heads: int, head_dim: int, wq, wk, eps: float, cos, sin):
     if rc:
         raise ValueError(f"orc_qkv_norm_rope: {rc}")
     return out
+
+
+def gelu_bf16(y) -> np.ndarray:
+    """bf16 bits of GELU (erf form) of the unrounded values y, one rounding."""
+    y = _c(y, np.float64)
+    h = np.zeros(y.shape, np.uint16)
+    lib().orc_gelu_bf16(_p(y), y.size, _p(h))
+    return h
+
+
+def mlp_gelu_down_act(prec, y_up, inv_lam_down, s_tx, L1_down):
+    """Fused GELU-MLP epilogue: the down-projection's activation-pass outputs
+    (codes, scales, P) from the up-projection's unrounded output."""
+    return quantize_act(prec, gelu_bf16(y_up), inv_lam_down, s_tx, L1_down)
 
 
 # ---------------------------------------------------------------- awq_w4a16

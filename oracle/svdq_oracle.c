@@ -576,6 +576,23 @@ int orc_qkv_norm_rope(int M, int H, int D, const double* y, const uint16_t* wq, 
 }
 
 /* ------------------------------------------------------------------------- */
+/* fused GELU-MLP epilogue                                                     */
+/* ------------------------------------------------------------------------- */
+/* The MLP's up-projection output y (unrounded, as the GEMM accumulator holds
+ * it) through GELU, rounded once to the bf16 activation the down-projection's
+ * activation pass reads (Diffusers "Nunchaku Lite" page, section on fused
+ * kernels: the MLP uses a fused GELU kernel):
+ *   h = bf16( y * (1 + erf(y / sqrt(2))) / 2 )
+ * in double. The down-projection then takes h through orc_svdq_quantize_act. */
+void orc_gelu_bf16(const double* y, int64_t n, uint16_t* h) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    const double v = y[i];
+    h[i] = orc_bf16_rn_f64(0.5 * v * (1.0 + erf(v * 0.70710678118654752440)));
+  }
+}
+
+/* ------------------------------------------------------------------------- */
 /* array forms of the format conversions (for the tests)                     */
 /* ------------------------------------------------------------------------- */
 

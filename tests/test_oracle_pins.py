@@ -618,3 +618,45 @@ def test_qkv_heads_and_sections_are_independent():
     assert np.array_equal(_heads(o3, 0), _heads(o, 0)) and not np.array_equal(_heads(o3, 1), _heads(o, 1))
     o4 = oracle.qkv_norm_rope(y, H_Q, D_Q, ONES, wk, 1e-6, c, s)
     assert np.array_equal(_heads(o4, 1), _heads(o, 1)) and not np.array_equal(_heads(o4, 0), _heads(o, 0))
+
+
+# ------------------------------------------------------------------ fused GELU-MLP epilogue
+def test_gelu_bf16_matches_scipy_erf_and_torch_rounding():
+    # an independent GELU (scipy's erf) rounded by torch's bfloat16 conversion
+    import scipy.special
+    rng = np.random.default_rng(21)
+    y = np.concatenate([rng.standard_normal(20000) * 3, rng.uniform(-12, 12, 5000), [0.0, 1e-30, -1e-30]])
+    ref = 0.5 * y * (1.0 + scipy.special.erf(y / np.sqrt(2.0)))
+    ref_bits = torch.from_numpy(ref).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.gelu_bf16(y)
+    # torch may round float64 -> bfloat16 through float32; that can only differ
+    # from one rounding where the float32 value sits exactly on a bf16 tie
+    low = ref.astype(np.float32).view(np.uint32) & 0xFFFF
+    safe = low != 0x8000
+    assert safe.mean() > 0.99
+    assert np.array_equal(got[safe], ref_bits[safe])
+
+
+def test_gelu_bf16_odd_part_identity_and_limits():
+    # GELU(x) - GELU(-x) = x for the Gaussian CDF; each side carries one bf16 rounding
+    x = np.random.default_rng(22).uniform(-8, 8, 4000)
+    gp = oracle.bf16_to_f32(oracle.gelu_bf16(x)).astype(np.float64)
+    gm = oracle.bf16_to_f32(oracle.gelu_bf16(-x)).astype(np.float64)
+    tol = (np.abs(gp) + np.abs(gm)) * 2.0 ** -8 + 1e-30
+    assert (np.abs(gp - gm - x) <= tol).all()
+    assert oracle.gelu_bf16(np.array([0.0]))[0] == 0
+    big = np.array([8.0, 20.0, 100.0])
+    assert np.array_equal(oracle.gelu_bf16(big), oracle.bf16_rn(big))
+    assert (np.abs(oracle.bf16_to_f32(oracle.gelu_bf16(-big))) < 1e-13).all()
+
+
+def test_mlp_epilogue_reduces_to_the_activation_pass_where_gelu_is_identity():
+    # for y >= 8, GELU(y) = y to well below a bf16 ulp, so the fused epilogue's
+    # down-projection inputs are those of the plain activation pass on bf16(y)
+    d = synth.svdq_layer(23, 6, 128, 8, 16)
+    y = 8.0 + np.abs(np.random.default_rng(23).standard_normal((6, 128))) * 4
+    for prec in ("nvfp4", "int4"):
+        a = oracle.mlp_gelu_down_act(prec, y, d["lam"] * 0 + 1.0, 1.0, d["L1"])
+        b = oracle.quantize_act(prec, oracle.bf16_rn(y), d["lam"] * 0 + 1.0, 1.0, d["L1"])
+        for k in ("codes", "scales", "P"):
+            assert np.array_equal(a[k], b[k])

@@ -72,3 +72,33 @@ def test_awq_ragged_shapes_with_bias(M, K, N):
     assert np.array_equal(w.q.cpu().numpy(), pk["q"])
     yo = oracle.awq_linear(d["x"], pk, b)
     check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
+
+
+def test_awq_chained_launches_read_the_previous_output():
+    """Three back-to-back launches on one stream, each reading the previous
+    one's output as its activations (no host synchronisation between them).
+    The launches may start before the previous one finishes, so this checks
+    that every launch waits for its input: each output must match the oracle
+    applied to the GPU's own previous output. The intermediate buffers start
+    as NaN, so a launch that read them early would not pass."""
+    M, K = 4, 512
+    ws, pks = [], []
+    for i in range(3):
+        d = synth.awq_inputs(40 + i, M, K, K, w_std=0.05)
+        ws.append(svdq.awq_pack_weight(torch.from_numpy(d["W"]).cuda()))
+        pks.append(oracle.awq_pack_weight(d["W"]))
+    x0 = synth.awq_inputs(39, M, K, K)["x"]
+    ys = [torch.full((M, K), float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    torch.cuda.synchronize()
+    inp = bf16_dev(x0)
+    for i in range(3):
+        svdq.awq_w4a16_linear(inp, ws[i], out=ys[i])
+        inp = ys[i]
+    torch.cuda.synchronize()
+    assert svdq.device_error() == 0
+    prev = x0
+    for i in range(3):
+        got = bf16_np(ys[i])
+        yo = oracle.awq_linear(prev, pks[i])
+        check_bf16_output(oracle.bf16_to_f32(got), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
+        prev = got

@@ -90,3 +90,19 @@ def test_validation_rejects_before_any_device_access(lib):
     assert lib.awq_w4a16_linear(0, 64, 8, None, None, None, None, None, None, None) == S.OK
     assert lib.awq_w4a16_linear(1, 64, 8, FAKE + 2, FAKE, FAKE, FAKE, None, FAKE, None) == S.ALIGN
     assert lib.svdq_probe_convert(None, 5, None, None, None, None) == S.INVALID_ARG
+
+
+def test_awq_rejects_k_beyond_the_shared_memory_bound(lib):
+    # the activations of a block of rows are held in shared memory: K <= 16384
+    assert lib.awq_w4a16_linear(1, 16384 + 64, 8, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == svdq.Status.SHAPE
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    # the binding passes device pointers only; a host or non-contiguous tensor
+    # is refused before anything reaches the library
+    import torch
+    with pytest.raises(ValueError, match="CUDA"):
+        svdq._ptr(torch.zeros(4))
+    if torch.cuda.is_available():
+        with pytest.raises(ValueError, match="contiguous"):
+            svdq._ptr(torch.zeros(4, 4, device="cuda").t())

@@ -45,3 +45,15 @@ def test_low_rank_factors_near_eckart_young():
     L2 = synth.bf16_bits_to_f32(d["L2"]).astype(np.float64)
     err = np.linalg.norm(What - L1 @ L2)
     assert best <= err <= best * 1.01
+
+
+def test_qkv_epilogue_inputs():
+    a = synth.qkv_epilogue_inputs(2, 64, 128, 24)
+    b = synth.qkv_epilogue_inputs(2, 64, 128, 24)
+    assert np.array_equal(a["wq"], b["wq"]) and not np.array_equal(a["wq"], a["wk"])
+    w = synth.bf16_bits_to_f32(a["wq"])
+    assert w.shape == (128,) and (w >= 0.5).all() and (w <= 1.5).all()
+    assert a["cos"].shape == (64, 64) and a["sin"].dtype == np.float32
+    # position 0 is not rotated; every (cos, sin) pair is a unit vector
+    assert (a["cos"][0] == 1).all() and (a["sin"][0] == 0).all()
+    assert np.allclose(a["cos"].astype(np.float64) ** 2 + a["sin"].astype(np.float64) ** 2, 1, atol=1e-6)

@@ -243,9 +243,10 @@ def run_cuda(args):
     step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
     k1_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
     k2_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
-    ms = max_over_ranks(world, statistics.mean(step_ms))
-    k1 = max_over_ranks(world, statistics.mean(k1_ms))
-    k2 = max_over_ranks(world, statistics.mean(k2_ms))
+    # the median of the timed steps (one slow step does not move it), max over ranks
+    ms = max_over_ranks(world, statistics.median(step_ms))
+    k1 = max_over_ranks(world, statistics.median(k1_ms))
+    k2 = max_over_ranks(world, statistics.median(k2_ms))
     flops = 2.0 * M * N * K
     value = whole_job_tflops(world, flops, ms)
 
@@ -257,6 +258,7 @@ def run_cuda(args):
     P = peaks()
     fp4_peak = P["bf16"] * NOMINAL_FP4_OVER_BF16
     k2_tflops = flops / (k2 * 1e-3) / 1e12
+    probe = mma_probe(svdq) if rank == 0 and not args.no_probe else None
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -277,12 +279,17 @@ def run_cuda(args):
                    "parallelism": f"{world} independent replicas (weak scaling, no collective)"},
         "pct_dense_fp4_peak_spec": round(100.0 * value / world / FP4_DENSE_SPEC_TFLOPS, 2),
         "kernels_ms": {"quantize_act": round(k1, 5), "w4a4_gemm": round(k2, 5)},
+        "step_ms_stats": {"median": round(statistics.median(step_ms), 5), "mean": round(statistics.mean(step_ms), 5),
+                          "min": round(min(step_ms), 5), "max": round(max(step_ms), 5), "n": len(step_ms),
+                          "statistic": "median of the timed steps (rank 0's spread shown)"},
         "roofline": {"kernel": "w4a4_gemm (tcgen05 mxf4nvf4)", "bound": "tensor",
                      "achieved": round(k2_tflops, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(k2_tflops / fp4_peak, 4),
                      "peak_source": f"{P['source']} bf16 burst {P['bf16']} x nominal fp4/bf16 ratio 4",
-                     "traffic": gemm_traffic()},
+                     "traffic": gemm_traffic(),
+                     "probe_peak": probe,
+                     "frac_of_probe": round(k2_tflops / probe["tflops"], 4) if probe else None},
         "e2e": {"value": round(whole_job_tflops(world, flops, e2e_ms), 3), "unit": "TFLOPS",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": round(e2e_ms, 4),
                 "overlap": "copy in, compute and copy out of consecutive steps on three streams, two device buffers"},
@@ -294,7 +301,7 @@ def run_cuda(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(d, rows=args.cpu_rows)
     if rank == 0 and not args.no_awq:
-        out["awq_gemv"] = bench_awq(svdq, P)
+        out["awq_gemv"] = [bench_awq(svdq, P, m) for m in synth.CONFIGS["c2_awq_gemv"]["Ms"]]
     if rank == 0 and not args.no_int4:
         out["int4_linear"] = bench_int4(svdq, P)
     if rank == 0:
@@ -303,6 +310,31 @@ def run_cuda(args):
         import torch.distributed as dist
 
         dist.destroy_process_group()
+
+
+def mma_probe(svdq, iters=4096, reps=5):
+    """The device's own rate for the GEMM's MMA instruction (block-scaled
+    NVFP4, 256 x 256 x 64 per CTA pair), from the library's probe kernel:
+    operands resident in shared memory, no loads, no epilogue. mode 0 = MMAs
+    only; mode 1 adds the GEMM's per-stage scale copies. Median of `reps`
+    launches timed with CUDA events."""
+    out = {}
+    for mode in (0, 1):
+        svdq.probe_mma_peak(iters, mode)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fl = svdq.probe_mma_peak(iters, mode)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        svdq.device_error()
+        out[f"mode{mode}"] = round(fl / (statistics.median(ts) * 1e-3) / 1e12, 1)
+    return {"tflops": out["mode0"], "tflops_with_scale_copies": out["mode1"], "unit": "TFLOP/s",
+            "what": "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 256x256x64 back to back on "
+                    "shared-memory operands, every SM pair (library probe kernel), median of 5 launches"}
 
 
 def e2e_pipelined(svdq, pw, L1, b, xh, M, N, K, steps, world):
@@ -371,7 +403,7 @@ def bench_int4(svdq, P, steps=10):
     y = svdq.w4a4_linear(qa, pw, b)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     ms = []
-    for i in range(steps + 2):
+    for i in range(steps + 3):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -379,10 +411,10 @@ def bench_int4(svdq, P, steps=10):
         svdq.w4a4_linear(qa, pw, b, out=y)
         e1.record()
         torch.cuda.synchronize()
-        if i >= 2:
+        if i >= 3:
             ms.append(e0.elapsed_time(e1))
     svdq.device_error()
-    t = statistics.mean(ms)
+    t = statistics.median(ms)
     tops = 2.0 * M * N * K / (t * 1e-3) / 1e12
     peak = P["bf16"] * NOMINAL_INT8_OVER_BF16
     return {"workload": f"svdq_w4a4 int4 g64 M{M} K{K} N{N} r{r}", "ms_per_step": round(t, 4),
@@ -391,20 +423,20 @@ def bench_int4(svdq, P, steps=10):
             "frac": round(tops / peak, 4), "steps": steps}
 
 
-def bench_awq(svdq, P):
-    """AWQ W4A16 GEMV (M = 1, K 3072, N 18432): HBM-bound. Weights rotate over
-    copies totalling > 3x L2 so every launch streams from HBM; the launches are
-    replayed from a CUDA graph, since one launch takes less device time than
-    the host needs to issue it."""
+def bench_awq(svdq, P, M=1):
+    """AWQ W4A16 modulation projection (M rows, K 3072, N 18432): HBM-bound at
+    small M. Weights rotate over copies totalling > 3x L2 so every launch
+    streams from HBM; the launches are replayed from a CUDA graph, since one
+    launch takes less device time than the host needs to issue it."""
     c = synth.CONFIGS["c2_awq_gemv"]
     K, N = c["K"], c["N"]
-    d = synth.awq_inputs(c["seed"], 1, K, N)
+    d = synth.awq_inputs(c["seed"], M, K, N)
     w0 = svdq.awq_pack_weight(torch.from_numpy(d["W"]).cuda())
     copies = []
     for _ in range(12):  # 12 x 31.9 MB = 383 MB
         copies.append(svdq.AwqWeight(K, N, w0.q.clone(), w0.scales.clone(), w0.zeros.clone()))
     x = bf16_dev(d["x"])
-    y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     side = torch.cuda.Stream()
     with torch.cuda.stream(side):
         for w in copies:
@@ -428,10 +460,11 @@ def bench_awq(svdq, P):
     svdq.device_error()
     launches = reps * rounds * len(copies)
     us = s.elapsed_time(e) * 1e3 / launches
-    byts = N * K // 2 + 2 * 2 * N * (K // 64) + K * 2 + N * 2
+    byts = N * K // 2 + 2 * 2 * N * (K // 64) + M * K * 2 + M * N * 2
     gbs = byts / (us * 1e-6) / 1e9
-    return {"M": 1, "K": K, "N": N, "us_per_launch": round(us, 3), "algorithmic_bytes": byts,
+    return {"M": M, "K": K, "N": N, "us_per_launch": round(us, 3), "algorithmic_bytes": byts,
             "achieved_gbs": round(gbs, 1), "peak_gbs": P["hbm_gbs"], "frac": round(gbs / P["hbm_gbs"], 4),
+            "tflops": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 3),
             "timing": f"CUDA graph of {rounds * len(copies)} launches over 12 rotating weight copies, replayed {reps}x"}
 
 
@@ -450,6 +483,53 @@ def cpu_baseline(d, rows: int, tag="oracle"):
     return {"value": round(2.0 * rows * N * K / dt / 1e12, 6), "unit": "TFLOPS", "cores": oracle.threads(),
             "kind": tag, "sample": f"first {min(rows, c['M'])} of {c['M']} rows of the workload (quantize_act + "
                                     "linear, float64 accumulation); weight pack untimed", "seconds": round(dt, 3)}
+
+
+def oracle_configs():
+    """Wall time of the CPU oracle on every workload, in full (the weight pack
+    untimed): svdq workloads = quantize_act + linear over all M rows; the AWQ
+    GEMV at each M of its sweep. The small workloads are also timed on one
+    thread. One JSON line; a reported baseline, not a target."""
+    import oracle
+
+    nthreads = oracle.threads()
+    out = {"kind": "oracle wall time per workload", "threads": nthreads, "nproc": os.cpu_count(), "workloads": {}}
+
+    def svdq_time(name, threads=None):
+        c = synth.CONFIGS[name]
+        d = synth.config_layer(name)
+        w = oracle.pack_weight(c["prec"], d["W"], d["lam"], d["L1"], d["L2"])
+        if threads:
+            oracle.set_threads(threads)
+        t0 = time.perf_counter()
+        a = oracle.quantize_act(c["prec"], d["x"], w["inv_lam"], 1.0, d["L1"])
+        oracle.linear(c["prec"], a, w, 1.0, d["L2"], d["b"])
+        dt = time.perf_counter() - t0
+        oracle.set_threads(nthreads)
+        return dt, 2.0 * c["M"] * c["N"] * c["K"]
+
+    for name in ("c1_smoke_nvfp4", "c3_qkv_nvfp4", "c4_mlp_up_nvfp4", "c4_mlp_down_nvfp4", "c5_qkv_int4"):
+        dt, fl = svdq_time(name)
+        e = {"seconds": round(dt, 3), "tflops": round(fl / dt / 1e12, 6), "threads": nthreads}
+        if name == "c1_smoke_nvfp4":
+            dt1, _ = svdq_time(name, threads=1)
+            e["seconds_1_thread"] = round(dt1, 3)
+        out["workloads"][name] = e
+    c = synth.CONFIGS["c2_awq_gemv"]
+    for m in c["Ms"]:
+        d = synth.awq_inputs(c["seed"], m, c["K"], c["N"])
+        pk = oracle.awq_pack_weight(d["W"])
+        t0 = time.perf_counter()
+        oracle.awq_linear(d["x"], pk)
+        dt = time.perf_counter() - t0
+        oracle.set_threads(1)
+        t0 = time.perf_counter()
+        oracle.awq_linear(d["x"], pk)
+        dt1 = time.perf_counter() - t0
+        oracle.set_threads(nthreads)
+        out["workloads"][f"c2_awq_gemv_m{m}"] = {"seconds": round(dt, 4), "seconds_1_thread": round(dt1, 4),
+                                                 "threads": nthreads}
+    print(json.dumps(out), flush=True)
 
 
 def run_reference(args):
@@ -473,7 +553,7 @@ def run_reference(args):
         oracle.linear("nvfp4", a, w, 1.0, d["L2"], d["b"])
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
-    s = statistics.mean(times)
+    s = statistics.median(times)
     value = 2.0 * rows * N * K / s / 1e12
     sample = f"{rows} rows per step of the M{M} K{K} N{N} r{r} workload (CPU oracle, float64 accumulation)"
     out = {
@@ -500,10 +580,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-awq", action="store_true")
     ap.add_argument("--no-int4", action="store_true")
+    ap.add_argument("--no-probe", action="store_true")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="only time the CPU oracle on every workload (no GPU needed) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.oracle_configs:
+        oracle_configs()
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_cuda(args)

@@ -29,7 +29,7 @@ __all__ = [
     "NVFP4", "INT4", "Status", "SvdqError", "PackedWeight", "QuantAct", "AwqWeight",
     "library_path", "load", "scale_bytes", "pack_weight", "quantize_act", "w4a4_linear",
     "svdq_linear", "awq_pack_weight", "awq_w4a16_linear", "device_error", "set_wait_limit_ns",
-    "probe_convert", "probe_wait_timeout", "debug_force_arch",
+    "probe_convert", "probe_wait_timeout", "probe_mma_peak", "debug_force_arch",
 ]
 
 NVFP4, INT4 = 0, 1
@@ -67,7 +67,7 @@ SIGNATURES = {
     "svdq_scale_bytes": (C.c_size_t, [_I, _I, _I]),
     "svdq_lr_up_elems": (C.c_size_t, [_I, _I, _I]),
     "svdq_pack_weight": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P]),
-    "svdq_quantize_act": (_I, [_I, _I, _I, _I, _P, _P, _F, _P, _P, _P, _P, _P]),
+    "svdq_quantize_act": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     "awq_pack_weight": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "awq_w4a16_linear": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
@@ -76,6 +76,7 @@ SIGNATURES = {
     "svdq_probe_convert": (_I, [_P, _I64, _P, _P, _P, _P]),
     "svdq_probe_wait_timeout": (_I, [_U64, _P]),
     "svdq_debug_force_arch": (None, [_I, _I]),
+    "svdq_probe_mma_peak": (_I, [_I, _I, _P]),
 }
 
 
@@ -109,7 +110,29 @@ def _ptr(t: Optional[torch.Tensor]):
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
     return t.data_ptr()
+
+
+def _need(cond: bool, what: str) -> None:
+    """Argument check of the binding: the C ABI receives bare pointers and
+    cannot see sizes, so every shape and dtype is checked here, before any
+    pointer reaches the library (a wrong size would otherwise become a read
+    or write past an allocation)."""
+    if not cond:
+        raise ValueError(what)
+
+
+def _is(t: Optional[torch.Tensor], dtype, shape, name: str) -> None:
+    _need(t is not None, f"{name}: missing")
+    _need(t.dtype == dtype, f"{name}: dtype {t.dtype}, expected {dtype}")
+    _need(tuple(t.shape) == tuple(shape), f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _at_least(t: torch.Tensor, dtype, nbytes: int, name: str) -> None:
+    _need(t.dtype == dtype, f"{name}: dtype {t.dtype}, expected {dtype}")
+    _need(t.numel() * t.element_size() >= nbytes, f"{name}: {t.numel() * t.element_size()} bytes, need {nbytes}")
 
 
 def _stream(stream=None):
@@ -152,12 +175,31 @@ class QuantAct:
     P: Optional[torch.Tensor]  # bf16 [M, r]
 
 
+def _check_packed(pw: PackedWeight) -> None:
+    """The buffers of a packed weight have the sizes its (prec, K, N, r) imply."""
+    _need(pw.prec in (NVFP4, INT4), f"precision {pw.prec!r}")
+    _is(pw.codes, torch.uint8, (pw.N, pw.K // 2), "pw.codes")
+    _at_least(pw.scales, torch.uint8, scale_bytes(pw.prec, pw.N, pw.K), "pw.scales")
+    _is(pw.tensor_scale, torch.float32, (2,), "pw.tensor_scale")
+    _is(pw.inv_lambda, torch.float32, (pw.K,), "pw.inv_lambda")
+    if pw.r:
+        _is(pw.lr_up, torch.bfloat16, (pw.N, 2 * pw.r if pw.prec == NVFP4 else pw.r), "pw.lr_up")
+
+
 def pack_weight(prec, W: torch.Tensor, lam: torch.Tensor, L1: Optional[torch.Tensor],
                 L2: Optional[torch.Tensor], act_tensor_scale: float = 1.0, stream=None) -> PackedWeight:
     """svdq_pack_weight: W fp32 [K, N], lam fp32 [K], L1 bf16 [K, r], L2 bf16 [r, N]."""
     p = _prec(prec)
+    _need(p in (NVFP4, INT4), f"precision {prec!r}")
+    _need(W.dim() == 2 and W.dtype == torch.float32, "W: expected float32 [K, N]")
     K, N = W.shape
     r = 0 if L1 is None else L1.shape[1]
+    _is(lam, torch.float32, (K,), "lambda")
+    if r:
+        _is(L1, torch.bfloat16, (K, r), "L1")
+        _is(L2, torch.bfloat16, (r, N), "L2")
+    else:
+        _need(L2 is None or L2.numel() == 0, "L2 given without L1")
     dev = W.device
     codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty(max(scale_bytes(p, N, K), 16), dtype=torch.uint8, device=dev)
@@ -173,16 +215,28 @@ def pack_weight(prec, W: torch.Tensor, lam: torch.Tensor, L1: Optional[torch.Ten
 
 def quantize_act(x: torch.Tensor, pw: PackedWeight, L1: Optional[torch.Tensor], stream=None,
                  out: Optional[QuantAct] = None) -> QuantAct:
-    """svdq_quantize_act: x bf16 [M, K] -> codes, scales, P."""
+    """svdq_quantize_act: x bf16 [M, K] -> codes, scales, P. The activation
+    tensor scale is the one packed into ``pw.tensor_scale`` (read on the device)."""
+    _need(x.dim() == 2 and x.dtype == torch.bfloat16, "x: expected bfloat16 [M, K]")
     M, K = x.shape
+    _check_packed(pw)
     p, r = pw.prec, pw.r
+    _need(K == pw.K, f"x has K = {K}, the packed weight K = {pw.K}")
+    if r:
+        _is(L1, torch.bfloat16, (K, r), "L1")
     dev = x.device
     if out is None:
         out = QuantAct(p, M, K, r, torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
                        torch.empty(max(scale_bytes(p, M, K), 16), dtype=torch.uint8, device=dev),
                        torch.empty((M, r), dtype=torch.bfloat16, device=dev) if r else None)
+    else:
+        _need((out.prec, out.M, out.K, out.r) == (p, M, K, r), "out: QuantAct of another shape or precision")
+        _is(out.codes, torch.uint8, (M, K // 2), "out.codes")
+        _at_least(out.scales, torch.uint8, scale_bytes(p, M, K), "out.scales")
+        if r:
+            _is(out.P, torch.bfloat16, (M, r), "out.P")
     _check("svdq_quantize_act", load().svdq_quantize_act(
-        p, M, K, r, _ptr(x), _ptr(pw.inv_lambda), float(pw.act_tensor_scale), _ptr(L1),
+        p, M, K, r, _ptr(x), _ptr(pw.inv_lambda), _ptr(pw.tensor_scale), _ptr(L1),
         _ptr(out.codes), _ptr(out.scales), _ptr(out.P), _stream(stream)))
     return out
 
@@ -191,6 +245,21 @@ def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = N
                 out_dtype: str = "bf16", stream=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """svdq_w4a4_linear: the 4-bit GEMM with the low-rank up-projection and bias fused."""
     M, K, N = qa.M, qa.K, pw.N
+    _check_packed(pw)
+    _need((qa.prec, qa.K, qa.r) == (pw.prec, pw.K, pw.r),
+          f"activations (prec {qa.prec}, K {qa.K}, r {qa.r}) do not match the weight "
+          f"(prec {pw.prec}, K {pw.K}, r {pw.r})")
+    _is(qa.codes, torch.uint8, (M, K // 2), "qa.codes")
+    _at_least(qa.scales, torch.uint8, scale_bytes(qa.prec, M, K), "qa.scales")
+    if qa.r:
+        _is(qa.P, torch.bfloat16, (M, qa.r), "qa.P")
+    if bias is not None:
+        _is(bias, torch.bfloat16, (N,), "bias")
+    _need(out_dtype in _OUT, f"out_dtype {out_dtype!r}")
+    want = {"bf16": (torch.bfloat16, (M, N)), "f32": (torch.float32, (M, N)),
+            "i32_groups": (torch.int32, (M, N, K // 64))}[out_dtype]
+    if out is not None:
+        _is(out, want[0], want[1], "out")
     if out is None:
         if out_dtype == "bf16":
             out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.codes.device)
@@ -220,20 +289,38 @@ class AwqWeight:
     zeros: torch.Tensor   # bf16 [N, K/64]
 
 
-def awq_pack_weight(W: torch.Tensor, stream=None) -> AwqWeight:
+def awq_pack_weight(W: torch.Tensor, stream=None, out: Optional[AwqWeight] = None) -> AwqWeight:
+    """awq_pack_weight: W fp32 [K, N] -> q, scales, zeros (into ``out``'s
+    buffers when given)."""
+    _need(W.dim() == 2 and W.dtype == torch.float32, "W: expected float32 [K, N]")
     K, N = W.shape
     dev = W.device
-    q = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
-    s = torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev)
-    z = torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev)
-    _check("awq_pack_weight", load().awq_pack_weight(K, N, _ptr(W), _ptr(q), _ptr(s), _ptr(z),
-                                                     _stream(stream)))
-    return AwqWeight(K, N, q, s, z)
+    if out is None:
+        out = AwqWeight(K, N, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                        torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev),
+                        torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev))
+    else:
+        _need((out.K, out.N) == (K, N), f"out: AwqWeight of K {out.K}, N {out.N}")
+        _is(out.q, torch.uint8, (N, K // 2), "out.q")
+        _is(out.scales, torch.bfloat16, (N, K // 64), "out.scales")
+        _is(out.zeros, torch.bfloat16, (N, K // 64), "out.zeros")
+    _check("awq_pack_weight", load().awq_pack_weight(K, N, _ptr(W), _ptr(out.q), _ptr(out.scales),
+                                                     _ptr(out.zeros), _stream(stream)))
+    return out
 
 
 def awq_w4a16_linear(x: torch.Tensor, w: AwqWeight, bias: Optional[torch.Tensor] = None, stream=None,
                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(x.dim() == 2 and x.dtype == torch.bfloat16, "x: expected bfloat16 [M, K]")
     M, K = x.shape
+    _need(K == w.K, f"x has K = {K}, the packed weight K = {w.K}")
+    _is(w.q, torch.uint8, (w.N, w.K // 2), "w.q")
+    _is(w.scales, torch.bfloat16, (w.N, w.K // 64), "w.scales")
+    _is(w.zeros, torch.bfloat16, (w.N, w.K // 64), "w.zeros")
+    if bias is not None:
+        _is(bias, torch.bfloat16, (w.N,), "bias")
+    if out is not None:
+        _is(out, torch.bfloat16, (M, w.N), "out")
     if out is None:
         out = torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
     _check("awq_w4a16_linear", load().awq_w4a16_linear(
@@ -269,6 +356,14 @@ def probe_convert(x: torch.Tensor, e2m1: bool = True, e4m3: bool = True, bf16: b
 
 def probe_wait_timeout(limit_ns: int, stream=None) -> None:
     _check("svdq_probe_wait_timeout", load().svdq_probe_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def probe_mma_peak(iters: int, mode: int = 0, stream=None) -> float:
+    """Launches the tensor-core rate probe; returns the FLOPs it performs (the
+    caller times it on its stream)."""
+    _check("svdq_probe_mma_peak", load().svdq_probe_mma_peak(int(iters), int(mode), _stream(stream)))
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return float(sms // 2) * iters * 4 * 2.0 * 256 * 256 * 64
 
 
 def debug_force_arch(major: int, minor: int = 0) -> None:

@@ -163,16 +163,17 @@ svdq_status svdq_pack_weight(svdq_precision p, int K, int N, int r, const float*
 }
 
 svdq_status svdq_quantize_act(svdq_precision p, int M, int K, int r, const uint16_t* x, const float* inv_lambda,
-                              float act_tensor_scale, const uint16_t* L1, uint8_t* x_codes, void* x_scales,
+                              const float* w_tensor_scale, const uint16_t* L1, uint8_t* x_codes, void* x_scales,
                               uint16_t* P, void* stream) {
   svdq_status st = check_common(p, K, r);
   if (st != SVDQ_OK) return st;
   if (M < 0) return SVDQ_ERR_INVALID_ARG;
-  if (p == SVDQ_NVFP4 && !(act_tensor_scale > 0.0f && act_tensor_scale < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!x || !inv_lambda || !x_codes || !x_scales) return SVDQ_ERR_INVALID_ARG;
+  if (p == SVDQ_NVFP4 && !w_tensor_scale) return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!L1 || !P)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(inv_lambda) || !aligned16(x_codes) || !aligned16(x_scales) ||
+      (p == SVDQ_NVFP4 && (reinterpret_cast<uintptr_t>(w_tensor_scale) & 7)) ||
       (r > 0 && (!aligned16(L1) || !aligned16(P))))
     return SVDQ_ERR_ALIGN;
   unsigned* err = nullptr;
@@ -184,7 +185,7 @@ svdq_status svdq_quantize_act(svdq_precision p, int M, int K, int r, const uint1
     if (cudaMemsetAsync(static_cast<uint8_t*>(x_scales) + rb * per_rb, 0, per_rb, s) != cudaSuccess)
       return SVDQ_ERR_CUDA;
   }
-  QuantActArgs a{x, inv_lambda, L1, x_codes, x_scales, P, M, K, r, act_tensor_scale};
+  QuantActArgs a{x, inv_lambda, L1, x_codes, x_scales, P, M, K, r, p == SVDQ_NVFP4 ? w_tensor_scale : nullptr};
   return from_cuda(launch_quant_act((int)p, a, err, g_wait_ns.load(), s));
 }
 
@@ -271,6 +272,15 @@ svdq_status svdq_probe_wait_timeout(unsigned long long limit_ns, void* stream) {
   svdq_status st = device_info(&err, nullptr);
   if (st != SVDQ_OK) return st;
   return from_cuda(launch_probe_wait(err, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
+svdq_status svdq_probe_mma_peak(int iters, int mode, void* stream) {
+  if (iters < 1 || iters > (1 << 20) || (mode != 0 && mode != 1)) return SVDQ_ERR_INVALID_ARG;
+  unsigned* err = nullptr;
+  int sms = 0;
+  svdq_status st = device_info(&err, &sms);
+  if (st != SVDQ_OK) return st;
+  return from_cuda(launch_probe_mma(iters, mode, sms, err, g_wait_ns.load(), static_cast<cudaStream_t>(stream)));
 }
 
 void svdq_debug_force_arch(int major, int minor) {

@@ -119,7 +119,17 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == kComputeWarps && lane == 0) {
+    // Before the previous kernel in the stream has finished, only hints: the
+    // tensor map and the first weight tiles are pulled towards L2. Any input
+    // (weights, scales, zero points, x, bias) may have been written by that
+    // kernel, so nothing is read into shared memory or registers until
+    // griddepcontrol.wait below has returned.
+    tma_prefetch_desc(&tm_q);
+    for (int c = 0; c < nst && c < kStagesA; ++c) tma_prefetch_l2_2d(&tm_q, c * (kStageK / 2), n0);
+  }
   __syncthreads();
+  grid_dependency_wait();
 
   if (warp == kComputeWarps) {
     // ------------------------------------------------------------ producer
@@ -131,20 +141,14 @@ awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, u
       tma_load_2d(base + s * kStageBytesA, &tm_q, &full[s], cc * (kStageK / 2), n0);
     };
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       // this CTA's rows of scales and zero points (contiguous: rows n0 ..
-      // n0 + rows - 1, 16-byte aligned) and the first weight stages: packed
-      // weights are never written by an earlier kernel, so they stream
-      // before the wait for the previous kernel in the stream
+      // n0 + rows - 1, 16-byte aligned), the activations (one bulk copy per
+      // row) and the first weight stages, which need no release
       const uint32_t sz_bytes = (uint32_t)(min(kRowsA, N - n0) * L.sz_pitch);
       mbar_expect_tx(xbar, (uint32_t)(M * 2 * K) + 2 * sz_bytes);
       bulk_load(base + L.off_s, a.s + (size_t)n0 * ng, sz_bytes, xbar);
       bulk_load(base + L.off_z, a.z + (size_t)n0 * ng, sz_bytes, xbar);
-      // the first stages need no release
       for (; c < nst && c < kStagesA; ++c) issue_stage(c);
-      // the activations may come from the previous kernel (one bulk copy per
-      // row); y is written only after they have arrived
-      grid_dependency_wait();
       for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
       for (; c < nst; ++c) {
         const int s = c % kStagesA;

@@ -16,7 +16,7 @@ struct QuantActArgs {
   void* scales;               // NVFP4 tiled e4m3 / INT4 bf16 [M, K/64]
   uint16_t* P;                // bf16 [M, r]
   int M, K, r;
-  float s_tx;
+  const float* tensor_scale;  // NVFP4: [2] = {s_tw, s_tx} (s_tx read on the device); INT4: unused
 };
 cudaError_t launch_quant_act(int prec, const QuantActArgs& a, unsigned* err, unsigned long long wait_ns,
                              cudaStream_t s);
@@ -83,6 +83,8 @@ cudaError_t launch_gemm_int4(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_probe_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3,
                                  uint16_t* bf16, cudaStream_t s);
 cudaError_t launch_probe_wait(unsigned* err, unsigned long long limit_ns, cudaStream_t s);
+cudaError_t launch_probe_mma(int iters, int mode, int num_sms, unsigned* err, unsigned long long wait_ns,
+                             cudaStream_t s);
 
 // Host helper: encode a 2-D tiled tensor map (driver entry point looked up at
 // run time; no link-time dependency on libcuda).

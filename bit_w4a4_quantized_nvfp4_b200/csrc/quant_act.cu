@@ -156,8 +156,9 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     *abort_flag = 0;
     fence_mbar_init();
   }
+  const float s_tx = PREC == 0 ? a.tensor_scale[1] : 1.0f;
   if (PREC == 0 && threadIdx.x < 256) {
-    const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), a.s_tx);
+    const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), s_tx);
     rtab[threadIdx.x] = d != 0.f ? make_float2(__frcp_rn(d), 0.f) : make_float2(0.f, 1.f);
   }
   __syncthreads();
@@ -199,7 +200,7 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   const int lr = rt * 16 + rl;                 // local row
   const int m = row0 + lr;
   const bool row_ok = m < M;
-  const float six_t = __fmul_rn(6.0f, a.s_tx);
+  const float six_t = __fmul_rn(6.0f, s_tx);
   // this lane's outputs, advanced by one chunk per step: codes of columns
   // c*256 + kp*64 + 32h .. +31, and the scale word (NVFP4: the 4 scales of
   // 64-column atom 4c + kp in row m; INT4: scale 4c + kp of row m)

@@ -29,7 +29,9 @@
  *   - SVDQ_ERR_CUDA reports a failed launch (cudaGetLastError after launch).
  *   - Kernels bound every wait on another warp or on the copy engine; a wait
  *     that runs out sets the device error word (svdq_device_error) instead of
- *     hanging.
+ *     hanging. There is ONE error word per device, shared by every stream and
+ *     every call on that device: after concurrent calls on several streams a
+ *     set bit cannot be attributed to one of them.
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - Packed 4-bit codes: element 2j of a row in the low nibble of byte j.
  */
@@ -120,14 +122,17 @@ svdq_status svdq_pack_weight(svdq_precision p, int K, int N, int r, const float*
  *   NVFP4: per 16-block: sf = e4m3(amax/(6*s_tx)), code = e2m1(x_hat * (1/(float(sf)*s_tx)))
  *   INT4:  per 64-block: s = bf16(amax/7), q = clamp(rne(x_hat/s), -8, 7)
  *   P[m,j] = bf16(sum_k x_hat[m,k] L1[k,j])      (fp32 accumulation)
- * In:  x bf16 [M, K]; inv_lambda fp32 [K] (from svdq_pack_weight);
- *      act_tensor_scale = s_tx, the value given to svdq_pack_weight (NVFP4);
- *      L1 bf16 [K, r].
+ * In:  x bf16 [M, K]; inv_lambda fp32 [K] and w_tensor_scale fp32 [2] (both
+ *      from svdq_pack_weight of the layer); L1 bf16 [K, r].
+ *      The activation tensor scale s_tx is read from w_tensor_scale[1] on the
+ *      device, so the activation pass and the GEMM (which folds s_tx into its
+ *      output scale and into lr_up) always use the one value given to
+ *      svdq_pack_weight. INT4 ignores w_tensor_scale (it may be NULL).
  * Out: x_codes u8 [M, K/2]; x_scales (svdq_scale_bytes(p, M, K) bytes);
  *      P bf16 [M, r].
  * Shapes: as svdq_pack_weight; M >= 0 (M = 0 is a no-op). */
 svdq_status svdq_quantize_act(svdq_precision p, int M, int K, int r, const uint16_t* x,
-                              const float* inv_lambda, float act_tensor_scale, const uint16_t* L1,
+                              const float* inv_lambda, const float* w_tensor_scale, const uint16_t* L1,
                               uint8_t* x_codes, void* x_scales, uint16_t* P, void* stream);
 
 /* svdq_w4a4_linear — the 4-bit GEMM with the low-rank up-projection and the
@@ -163,7 +168,12 @@ svdq_status awq_pack_weight(int K, int N, const float* W, uint8_t* q, uint16_t* 
  * In:  x bf16 [M, K]; q, scales, zeros from awq_pack_weight; bias bf16 [N] or NULL.
  * Out: y bf16 [M, N].
  * Shapes: K % 64 == 0, K <= 16384 (the activations of a block of rows are
- * held in shared memory), N % 8 == 0, M >= 0. */
+ * held in shared memory), N % 8 == 0, M >= 0.
+ * Launched with programmatic dependent launch: the kernel may be scheduled
+ * while the previous kernel in the stream finishes, but it reads none of its
+ * inputs (x, q, scales, zeros, bias) before that kernel has completed, so any
+ * of them may be that kernel's output (e.g. awq_pack_weight into the same
+ * buffers just before). */
 svdq_status awq_w4a16_linear(int M, int K, int N, const uint16_t* x, const uint8_t* q,
                              const uint16_t* scales, const uint16_t* zeros, const uint16_t* bias,
                              uint16_t* y, void* stream);
@@ -192,6 +202,15 @@ svdq_status svdq_probe_convert(const float* in, long long n, uint8_t* e2m1, uint
  * `limit_ns`; it must set the timeout bit of the device error word and exit.
  * Exercises the bounded-wait path without hanging the GPU. */
 svdq_status svdq_probe_wait_timeout(unsigned long long limit_ns, void* stream);
+
+/* Tensor-core rate probe (the measured denominator of the GEMM's roofline):
+ * every CTA pair of the device (one pair per two SMs) issues `iters` K stages
+ * of 4 block-scaled NVFP4 MMAs (tcgen05.mma.cta_group::2.kind::mxf4nvf4,
+ * 256 x 256 x 64 each, the GEMM's instruction) on operands that stay in
+ * shared memory: no loads, no epilogue. mode 1 also issues the GEMM's 12
+ * scale copies (tcgen05.cp) per stage. The caller times the launch; the work
+ * is (SMs/2) * iters * 4 * 2*256*256*64 FLOP. 1 <= iters <= 2^20. */
+svdq_status svdq_probe_mma_peak(int iters, int mode, void* stream);
 
 /* Test hook: pretend the device has compute capability major.minor (0, 0
  * restores the real query), to exercise SVDQ_ERR_UNSUPPORTED_ARCH. */

@@ -71,11 +71,14 @@ def test_validation_rejects_before_any_device_access(lib):
     assert lib.svdq_pack_weight(0, 64, 8, 16, FAKE, FAKE, None, FAKE, 1.0, FAKE, FAKE, FAKE, FAKE, FAKE, None) == S.INVALID_ARG
     assert lib.svdq_pack_weight(0, 64, 8, 0, FAKE, FAKE, None, None, 0.0, FAKE, FAKE, FAKE, FAKE, None, None) == S.INVALID_ARG
     assert lib.svdq_pack_weight(0, 64, 8, 0, FAKE + 4, FAKE, None, None, 1.0, FAKE, FAKE, FAKE, FAKE, None, None) == S.ALIGN
-    # quantize
-    assert lib.svdq_quantize_act(0, -1, 64, 0, FAKE, FAKE, 1.0, None, FAKE, FAKE, None, None) == S.INVALID_ARG
-    assert lib.svdq_quantize_act(0, 0, 64, 0, None, None, 1.0, None, None, None, None, None) == S.OK  # M = 0 no-op
-    assert lib.svdq_quantize_act(1, 4, 96, 0, FAKE, FAKE, 1.0, None, FAKE, FAKE, None, None) == S.SHAPE
-    assert lib.svdq_quantize_act(0, 4, 64, 16, FAKE, FAKE, 1.0, FAKE, FAKE, FAKE, FAKE + 8, None) == S.ALIGN
+    # quantize (the 7th argument is the packed weight's tensor scales {s_tw, s_tx})
+    assert lib.svdq_quantize_act(0, -1, 64, 0, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None) == S.INVALID_ARG
+    assert lib.svdq_quantize_act(0, 0, 64, 0, None, None, None, None, None, None, None, None) == S.OK  # M = 0 no-op
+    assert lib.svdq_quantize_act(1, 4, 96, 0, FAKE, FAKE, None, None, FAKE, FAKE, None, None) == S.SHAPE
+    assert lib.svdq_quantize_act(0, 4, 64, 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, None) == S.ALIGN
+    # NVFP4 needs the tensor scales (s_tx is read from them); INT4 does not
+    assert lib.svdq_quantize_act(0, 4, 64, 0, FAKE, FAKE, None, None, FAKE, FAKE, None, None) == S.INVALID_ARG
+    assert lib.svdq_quantize_act(0, 4, 64, 0, FAKE, FAKE, FAKE + 4, None, FAKE, FAKE, None, None) == S.ALIGN
     # linear
     assert lib.svdq_w4a4_linear(0, 4, 64, 8, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, 2, None) == S.INVALID_ARG
     assert lib.svdq_w4a4_linear(0, 4, 64, 8, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, 9, None) == S.INVALID_ARG
@@ -106,3 +109,97 @@ def test_binding_refuses_host_and_strided_tensors():
     if torch.cuda.is_available():
         with pytest.raises(ValueError, match="contiguous"):
             svdq._ptr(torch.zeros(4, 4, device="cuda").t())
+
+
+# ------------------------------------------------------------------ binding argument checks
+# The C ABI sees bare pointers, so the binding checks every shape, dtype and
+# device before a pointer reaches the library. These run on CPU tensors: a
+# mismatch must raise ValueError naming the argument; a well-formed call gets
+# as far as the device check ("expected a CUDA tensor") and no further.
+import torch  # noqa: E402
+
+
+def _bf16(*shape):
+    return torch.zeros(shape, dtype=torch.bfloat16)
+
+
+def _packed(prec=svdq.NVFP4, K=128, N=16, r=16):
+    scales = torch.zeros(max(svdq.scale_bytes(prec, N, K), 16), dtype=torch.uint8)
+    lr = _bf16(N, 2 * r if prec == svdq.NVFP4 else r) if r else None
+    return svdq.PackedWeight(prec, K, N, r, torch.zeros((N, K // 2), dtype=torch.uint8), scales,
+                             torch.ones(2), torch.ones(K), lr, 1.0)
+
+
+def _act(prec=svdq.NVFP4, M=8, K=128, r=16):
+    return svdq.QuantAct(prec, M, K, r, torch.zeros((M, K // 2), dtype=torch.uint8),
+                         torch.zeros(max(svdq.scale_bytes(prec, M, K), 16), dtype=torch.uint8),
+                         _bf16(M, r) if r else None)
+
+
+def _raises(match, fn, *a, **kw):
+    with pytest.raises(ValueError, match=match):
+        fn(*a, **kw)
+
+
+def test_binding_checks_quantize_act(lib):
+    pw = _packed()
+    L1 = _bf16(128, 16)
+    _raises("CUDA", svdq.quantize_act, _bf16(8, 128), pw, L1)            # well formed
+    _raises("x: expected", svdq.quantize_act, torch.zeros(8, 128), pw, L1)
+    _raises("K = 64", svdq.quantize_act, _bf16(8, 64), pw, L1)
+    _raises("L1: shape", svdq.quantize_act, _bf16(8, 128), pw, _bf16(128, 32))
+    _raises("L1: dtype", svdq.quantize_act, _bf16(8, 128), pw, torch.zeros(128, 16))
+    bad = _packed()
+    bad.inv_lambda = torch.ones(64)
+    _raises("pw.inv_lambda", svdq.quantize_act, _bf16(8, 128), bad, L1)
+    bad = _packed()
+    bad.tensor_scale = torch.ones(1)
+    _raises("pw.tensor_scale", svdq.quantize_act, _bf16(8, 128), bad, L1)
+    out = _act(M=8)
+    out.codes = torch.zeros((8, 32), dtype=torch.uint8)
+    _raises("out.codes", svdq.quantize_act, _bf16(8, 128), pw, L1, out=out)
+    out = _act(M=8)
+    out.scales = torch.zeros(16, dtype=torch.uint8)
+    _raises("out.scales", svdq.quantize_act, _bf16(8, 128), pw, L1, out=out)
+    _raises("another shape", svdq.quantize_act, _bf16(8, 128), pw, L1, out=_act(M=4))
+
+
+def test_binding_checks_w4a4_linear(lib):
+    pw, qa = _packed(), _act()
+    _raises("CUDA", svdq.w4a4_linear, qa, pw)                            # well formed
+    _raises("do not match", svdq.w4a4_linear, _act(K=256), pw)
+    _raises("do not match", svdq.w4a4_linear, _act(prec=svdq.INT4), pw)
+    _raises("do not match", svdq.w4a4_linear, _act(r=0), pw)
+    _raises("bias: shape", svdq.w4a4_linear, qa, pw, _bf16(8))
+    _raises("bias: dtype", svdq.w4a4_linear, qa, pw, torch.zeros(16))
+    _raises("out: shape", svdq.w4a4_linear, qa, pw, out=_bf16(8, 8))
+    _raises("out: dtype", svdq.w4a4_linear, qa, pw, out=torch.zeros(8, 16))
+    _raises("out: shape", svdq.w4a4_linear, qa, pw, out_dtype="f32", out=torch.zeros(8, 8))
+    bad = _packed()
+    bad.codes = torch.zeros((16, 32), dtype=torch.uint8)
+    _raises("pw.codes", svdq.w4a4_linear, qa, bad)
+    bad = _packed()
+    bad.lr_up = _bf16(16, 16)
+    _raises("pw.lr_up", svdq.w4a4_linear, qa, bad)
+    bad = _act()
+    bad.P = _bf16(8, 8)
+    _raises("qa.P", svdq.w4a4_linear, bad, pw)
+    _raises("out_dtype", svdq.w4a4_linear, qa, pw, out_dtype="f16")
+
+
+def test_binding_checks_pack_and_awq(lib):
+    W = torch.zeros(128, 16)
+    _raises("CUDA", svdq.pack_weight, "nvfp4", W, torch.ones(128), _bf16(128, 16), _bf16(16, 16))
+    _raises("W: expected", svdq.pack_weight, "nvfp4", W.double(), torch.ones(128), None, None)
+    _raises("lambda: shape", svdq.pack_weight, "nvfp4", W, torch.ones(64), None, None)
+    _raises("L2: shape", svdq.pack_weight, "nvfp4", W, torch.ones(128), _bf16(128, 16), _bf16(16, 8))
+    _raises("precision", svdq.pack_weight, 5, W, torch.ones(128), None, None)
+    aw = svdq.AwqWeight(128, 16, torch.zeros((16, 64), dtype=torch.uint8), _bf16(16, 2), _bf16(16, 2))
+    _raises("CUDA", svdq.awq_w4a16_linear, _bf16(1, 128), aw)            # well formed
+    _raises("K = 64", svdq.awq_w4a16_linear, _bf16(1, 64), aw)
+    _raises("x: expected", svdq.awq_w4a16_linear, torch.zeros(1, 128), aw)
+    _raises("bias: shape", svdq.awq_w4a16_linear, _bf16(1, 128), aw, _bf16(8))
+    _raises("out: shape", svdq.awq_w4a16_linear, _bf16(2, 128), aw, out=_bf16(1, 16))
+    bad = svdq.AwqWeight(128, 16, torch.zeros((16, 64), dtype=torch.uint8), _bf16(16, 1), _bf16(16, 2))
+    _raises("w.scales", svdq.awq_w4a16_linear, _bf16(1, 128), bad)
+    _raises("W: expected", svdq.awq_pack_weight, torch.zeros(128, 16, dtype=torch.float64))

@@ -102,3 +102,38 @@ def test_awq_chained_launches_read_the_previous_output():
         yo = oracle.awq_linear(prev, pks[i])
         check_bf16_output(oracle.bf16_to_f32(got), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
         prev = got
+
+
+def test_awq_reads_weights_written_just_before():
+    """The GEMV may be scheduled before the previous kernel in the stream
+    finishes (dependent launch), so it must read none of its inputs early.
+    Two cases, each with no host synchronisation between the writer and the
+    GEMV: awq_pack_weight of a new weight into the buffers of an old one, and
+    a device copy of pre-packed tensors into those buffers (as a checkpoint
+    load would do). Each output must match the new weight."""
+    c = synth.CONFIGS["c2_awq_gemv"]
+    K, N = c["K"], c["N"]
+    old = synth.awq_inputs(50, 2, K, N)
+    new = synth.awq_inputs(51, 2, K, N, w_std=0.05)
+    pk_new = oracle.awq_pack_weight(new["W"])
+    yo = oracle.awq_linear(new["x"], pk_new)
+    x = bf16_dev(new["x"])
+    Wn = torch.from_numpy(new["W"]).cuda()
+
+    w = svdq.awq_pack_weight(torch.from_numpy(old["W"]).cuda())
+    torch.cuda.synchronize()
+    svdq.awq_pack_weight(Wn, out=w)
+    y = svdq.awq_w4a16_linear(x, w)
+    torch.cuda.synchronize()
+    assert svdq.device_error() == 0
+    check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
+
+    src = svdq.awq_pack_weight(Wn)
+    svdq.awq_pack_weight(torch.from_numpy(old["W"]).cuda(), out=w)
+    torch.cuda.synchronize()
+    w.q.copy_(src.q)
+    w.scales.copy_(src.scales)
+    w.zeros.copy_(src.zeros)
+    y2 = svdq.awq_w4a16_linear(x, w)
+    torch.cuda.synchronize()
+    check_bf16_output(oracle.bf16_to_f32(bf16_np(y2)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))

@@ -164,17 +164,48 @@ def test_zero_residual_gpu():
     check_bf16_output(as_f32(bf16_np(y)), yo, as_f32(oracle.bf16_rn(yo)))
 
 
-def test_c3_full_size_sampled_rows():
-    """The benchmark's workload (M4608 K3072 N9216 r32) in the benchmark's
-    launch configuration: codes and scales compared in full, y on 192 seeded
-    rows (the oracle computes those one by one)."""
-    c = dict(synth.CONFIGS["c3_qkv_nvfp4"])
-    d = synth.config_layer("c3_qkv_nvfp4")
+@pytest.mark.parametrize("name", ["c3_qkv_nvfp4", "c4_mlp_up_nvfp4", "c4_mlp_down_nvfp4"])
+def test_full_size_workload_sampled_rows(name):
+    """The full-size NVFP4 workloads in the benchmark's launch configuration:
+    the fused-QKV projection (M4608 K3072 N9216, the benchmark's workload) and
+    both projections of the MLP pair (4608x3072 -> 12288 and, on GELU inputs,
+    4608x12288 -> 3072; the K = 12288 activation pass walks 48 chunks, four
+    times the QKV's). Weight and activation codes and scales and P are compared
+    in full, y on 160 seeded rows (the oracle computes those one by one)."""
+    c = dict(synth.CONFIGS[name])
+    d = synth.config_layer(name)
     pw, qa, y = run_layer("nvfp4", d)
-    rows = np.sort(np.random.default_rng(3).choice(c["M"], 192, replace=False)).astype(np.int32)
+    rows = np.sort(np.random.default_rng(3).choice(c["M"], 160, replace=False)).astype(np.int32)
     w, a, yo = oracle_layer("nvfp4", d, rows=rows)
     compare_pack_and_act("nvfp4", d, pw, qa, w, a)
     check_bf16_output(as_f32(bf16_np(y))[rows], yo, as_f32(oracle.bf16_rn(yo)))
+
+
+@pytest.mark.parametrize("prec,M,K,r", [("nvfp4", 100, 320, 16), ("nvfp4", 33, 1024, 32), ("int4", 70, 192, 32)])
+def test_activation_pass_writes_nothing_past_its_outputs(prec, M, K, r):
+    """Every output of the activation pass (codes, scales, P) lives in a larger
+    buffer filled with a sentinel; after the pass the bytes past each output's
+    end still hold it, and the outputs match the oracle (ragged M and K)."""
+    d = synth.svdq_layer(27, M, K, 64, r)
+    W = torch.from_numpy(d["W"]).cuda()
+    lam = torch.from_numpy(d["lam"]).cuda()
+    L1, L2 = bf16_dev(d["L1"]), bf16_dev(d["L2"])
+    pw = svdq.pack_weight(prec, W, lam, L1, L2)
+    pad = 4096
+    nc, ns = M * K // 2, svdq.scale_bytes(prec, M, K)
+    codes = torch.full((nc + pad,), 0xA5, dtype=torch.uint8, device="cuda")
+    scales = torch.full((ns + pad,), 0x5A, dtype=torch.uint8, device="cuda")
+    P = torch.full((M * r + pad,), -777.0, dtype=torch.bfloat16, device="cuda")
+    out = svdq.QuantAct(pw.prec, M, K, r, codes[:nc].view(M, K // 2), scales[:ns], P[: M * r].view(M, r))
+    svdq.quantize_act(bf16_dev(d["x"]), pw, L1, out=out)
+    torch.cuda.synchronize()
+    assert svdq.device_error() == 0
+    assert (codes[nc:] == 0xA5).all(), "write past the end of the codes"
+    assert (scales[ns:] == 0x5A).all(), "write past the end of the scales"
+    assert (P[M * r:] == -777.0).all(), "write past the end of P"
+    w = oracle.pack_weight(prec, d["W"], d["lam"], d["L1"], d["L2"])
+    a = oracle.quantize_act(prec, d["x"], w["inv_lam"], 1.0, d["L1"])
+    compare_pack_and_act(prec, d, pw, out, w, a)
 
 
 # ------------------------------------------------------------------ INT4 (activation and pack side)

@@ -285,17 +285,21 @@ def _bf16_exact(q: Fraction) -> int:
     return best[1]
 
 
-@pytest.mark.parametrize("prec", ["nvfp4", "int4"])
-def test_linear_exact_on_tiny_problem(prec):
+@pytest.mark.parametrize("prec,s_tx", [("nvfp4", 1.0), ("nvfp4", 0.25), ("nvfp4", 0.7), ("int4", 1.0)])
+def test_linear_exact_on_tiny_problem(prec, s_tx):
+    """y = s_tx s_tw sum_b sx sw sum qx qw + P L2 + b, exactly in rationals from
+    the packed codes and scales. With s_tx != 1 an oracle that dropped s_tx
+    from the output scale (or applied it twice) fails here."""
     M, K, N, r = 4, 128, 8, 16
     d = synth.svdq_layer(7, M, K, N, r, x_out_frac=0.05, x_out_scale=10.0)
     w = oracle.pack_weight(prec, d["W"], d["lam"], d["L1"], d["L2"])
-    a = oracle.quantize_act(prec, d["x"], w["inv_lam"], 1.0, d["L1"])
-    y = oracle.linear(prec, a, w, 1.0, d["L2"], d["b"])
+    a = oracle.quantize_act(prec, d["x"], w["inv_lam"], s_tx, d["L1"])
+    y = oracle.linear(prec, a, w, s_tx, d["L2"], d["b"])
 
     xd = _deq_rows(prec, a["codes"], a["scales"])
     wd = _deq_rows(prec, w["codes"], w["scales"])
-    alpha = Fraction(w["s_tw"]) if prec == "nvfp4" else Fraction(1)
+    # s_tx is an fp32 value at every interface (the tensor-scale buffer)
+    alpha = Fraction(float(np.float32(s_tx))) * Fraction(w["s_tw"]) if prec == "nvfp4" else Fraction(1)
     P = [[Fraction(float(v)) for v in row] for row in oracle.bf16_to_f32(a["P"])]
     L2 = [[Fraction(float(v)) for v in row] for row in oracle.bf16_to_f32(d["L2"])]
     b = [Fraction(float(v)) for v in oracle.bf16_to_f32(d["b"])]

@@ -103,36 +103,57 @@ def _check(fn: str, status: int) -> None:
         raise SvdqError(fn, status, load().svdq_status_str(status).decode())
 
 
-def _ptr(t: Optional[torch.Tensor]):
+def _ptr(t: Optional[torch.Tensor], dev: Optional[int] = None):
+    """Device address of a contiguous CUDA tensor on the current device
+    (``dev``, when the caller has already read it)."""
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
-    if t.device.index != torch.cuda.current_device():
-        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+    cur = torch.cuda.current_device() if dev is None else dev
+    if t.get_device() != cur:
+        raise ValueError(f"tensor on {t.device}, but the current device is cuda:{cur}")
     return t.data_ptr()
 
 
-def _need(cond: bool, what: str) -> None:
+def _ptrs(*ts):
+    """_ptr of several tensors, reading the current device once."""
+    dev = None
+    out = []
+    for t in ts:
+        if t is not None and dev is None:
+            if not t.is_cuda:
+                raise ValueError("expected a CUDA tensor")
+            dev = torch.cuda.current_device()
+        out.append(_ptr(t, dev))
+    return out
+
+
+def _need(cond: bool, what, *args) -> None:
     """Argument check of the binding: the C ABI receives bare pointers and
     cannot see sizes, so every shape and dtype is checked here, before any
     pointer reaches the library (a wrong size would otherwise become a read
-    or write past an allocation)."""
+    or write past an allocation). The message is formatted only on failure."""
     if not cond:
-        raise ValueError(what)
+        raise ValueError(what.format(*args) if args else what)
 
 
 def _is(t: Optional[torch.Tensor], dtype, shape, name: str) -> None:
-    _need(t is not None, f"{name}: missing")
-    _need(t.dtype == dtype, f"{name}: dtype {t.dtype}, expected {dtype}")
-    _need(tuple(t.shape) == tuple(shape), f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t is None:
+        raise ValueError(f"{name}: missing")
+    if t.dtype is not dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.shape != shape:
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
 def _at_least(t: torch.Tensor, dtype, nbytes: int, name: str) -> None:
-    _need(t.dtype == dtype, f"{name}: dtype {t.dtype}, expected {dtype}")
-    _need(t.numel() * t.element_size() >= nbytes, f"{name}: {t.numel() * t.element_size()} bytes, need {nbytes}")
+    if t.dtype is not dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name}: {t.numel() * t.element_size()} bytes, need {nbytes}")
 
 
 def _stream(stream=None):
@@ -177,7 +198,7 @@ class QuantAct:
 
 def _check_packed(pw: PackedWeight) -> None:
     """The buffers of a packed weight have the sizes its (prec, K, N, r) imply."""
-    _need(pw.prec in (NVFP4, INT4), f"precision {pw.prec!r}")
+    _need(pw.prec in (NVFP4, INT4), "precision {!r}", pw.prec)
     _is(pw.codes, torch.uint8, (pw.N, pw.K // 2), "pw.codes")
     _at_least(pw.scales, torch.uint8, scale_bytes(pw.prec, pw.N, pw.K), "pw.scales")
     _is(pw.tensor_scale, torch.float32, (2,), "pw.tensor_scale")
@@ -190,7 +211,7 @@ def pack_weight(prec, W: torch.Tensor, lam: torch.Tensor, L1: Optional[torch.Ten
                 L2: Optional[torch.Tensor], act_tensor_scale: float = 1.0, stream=None) -> PackedWeight:
     """svdq_pack_weight: W fp32 [K, N], lam fp32 [K], L1 bf16 [K, r], L2 bf16 [r, N]."""
     p = _prec(prec)
-    _need(p in (NVFP4, INT4), f"precision {prec!r}")
+    _need(p in (NVFP4, INT4), "precision {!r}", prec)
     _need(W.dim() == 2 and W.dtype == torch.float32, "W: expected float32 [K, N]")
     K, N = W.shape
     r = 0 if L1 is None else L1.shape[1]
@@ -221,7 +242,7 @@ def quantize_act(x: torch.Tensor, pw: PackedWeight, L1: Optional[torch.Tensor], 
     M, K = x.shape
     _check_packed(pw)
     p, r = pw.prec, pw.r
-    _need(K == pw.K, f"x has K = {K}, the packed weight K = {pw.K}")
+    _need(K == pw.K, "x has K = {}, the packed weight K = {}", K, pw.K)
     if r:
         _is(L1, torch.bfloat16, (K, r), "L1")
     dev = x.device
@@ -230,14 +251,14 @@ def quantize_act(x: torch.Tensor, pw: PackedWeight, L1: Optional[torch.Tensor], 
                        torch.empty(max(scale_bytes(p, M, K), 16), dtype=torch.uint8, device=dev),
                        torch.empty((M, r), dtype=torch.bfloat16, device=dev) if r else None)
     else:
-        _need((out.prec, out.M, out.K, out.r) == (p, M, K, r), "out: QuantAct of another shape or precision")
+        _need(out.prec == p and out.M == M and out.K == K and out.r == r,
+              "out: QuantAct of another shape or precision")
         _is(out.codes, torch.uint8, (M, K // 2), "out.codes")
         _at_least(out.scales, torch.uint8, scale_bytes(p, M, K), "out.scales")
         if r:
             _is(out.P, torch.bfloat16, (M, r), "out.P")
-    _check("svdq_quantize_act", load().svdq_quantize_act(
-        p, M, K, r, _ptr(x), _ptr(pw.inv_lambda), _ptr(pw.tensor_scale), _ptr(L1),
-        _ptr(out.codes), _ptr(out.scales), _ptr(out.P), _stream(stream)))
+    px, pil, pts, pl1, pc, psc, pp = _ptrs(x, pw.inv_lambda, pw.tensor_scale, L1, out.codes, out.scales, out.P)
+    _check("svdq_quantize_act", load().svdq_quantize_act(p, M, K, r, px, pil, pts, pl1, pc, psc, pp, _stream(stream)))
     return out
 
 
@@ -246,16 +267,16 @@ def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = N
     """svdq_w4a4_linear: the 4-bit GEMM with the low-rank up-projection and bias fused."""
     M, K, N = qa.M, qa.K, pw.N
     _check_packed(pw)
-    _need((qa.prec, qa.K, qa.r) == (pw.prec, pw.K, pw.r),
-          f"activations (prec {qa.prec}, K {qa.K}, r {qa.r}) do not match the weight "
-          f"(prec {pw.prec}, K {pw.K}, r {pw.r})")
+    _need(qa.prec == pw.prec and qa.K == pw.K and qa.r == pw.r,
+          "activations (prec {}, K {}, r {}) do not match the weight (prec {}, K {}, r {})",
+          qa.prec, qa.K, qa.r, pw.prec, pw.K, pw.r)
     _is(qa.codes, torch.uint8, (M, K // 2), "qa.codes")
     _at_least(qa.scales, torch.uint8, scale_bytes(qa.prec, M, K), "qa.scales")
     if qa.r:
         _is(qa.P, torch.bfloat16, (M, qa.r), "qa.P")
     if bias is not None:
         _is(bias, torch.bfloat16, (N,), "bias")
-    _need(out_dtype in _OUT, f"out_dtype {out_dtype!r}")
+    _need(out_dtype in _OUT, "out_dtype {!r}", out_dtype)
     want = {"bf16": (torch.bfloat16, (M, N)), "f32": (torch.float32, (M, N)),
             "i32_groups": (torch.int32, (M, N, K // 64))}[out_dtype]
     if out is not None:
@@ -267,10 +288,9 @@ def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = N
             out = torch.empty((M, N), dtype=torch.float32, device=qa.codes.device)
         else:
             out = torch.empty((M, N, K // 64), dtype=torch.int32, device=qa.codes.device)
-    _check("svdq_w4a4_linear", load().svdq_w4a4_linear(
-        pw.prec, M, K, N, pw.r, _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.P), _ptr(pw.codes),
-        _ptr(pw.scales), _ptr(pw.tensor_scale), _ptr(pw.lr_up), _ptr(bias), _ptr(out),
-        _OUT[out_dtype], _stream(stream)))
+    ptrs = _ptrs(qa.codes, qa.scales, qa.P, pw.codes, pw.scales, pw.tensor_scale, pw.lr_up, bias, out)
+    _check("svdq_w4a4_linear", load().svdq_w4a4_linear(pw.prec, M, K, N, pw.r, *ptrs, _OUT[out_dtype],
+                                                       _stream(stream)))
     return out
 
 
@@ -300,7 +320,7 @@ def awq_pack_weight(W: torch.Tensor, stream=None, out: Optional[AwqWeight] = Non
                         torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev),
                         torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev))
     else:
-        _need((out.K, out.N) == (K, N), f"out: AwqWeight of K {out.K}, N {out.N}")
+        _need(out.K == K and out.N == N, "out: AwqWeight of K {}, N {}", out.K, out.N)
         _is(out.q, torch.uint8, (N, K // 2), "out.q")
         _is(out.scales, torch.bfloat16, (N, K // 64), "out.scales")
         _is(out.zeros, torch.bfloat16, (N, K // 64), "out.zeros")
@@ -313,7 +333,7 @@ def awq_w4a16_linear(x: torch.Tensor, w: AwqWeight, bias: Optional[torch.Tensor]
                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
     _need(x.dim() == 2 and x.dtype == torch.bfloat16, "x: expected bfloat16 [M, K]")
     M, K = x.shape
-    _need(K == w.K, f"x has K = {K}, the packed weight K = {w.K}")
+    _need(K == w.K, "x has K = {}, the packed weight K = {}", K, w.K)
     _is(w.q, torch.uint8, (w.N, w.K // 2), "w.q")
     _is(w.scales, torch.bfloat16, (w.N, w.K // 64), "w.scales")
     _is(w.zeros, torch.bfloat16, (w.N, w.K // 64), "w.zeros")

@@ -82,31 +82,117 @@ EncodeFn encode_fn() {
 }
 }  // namespace
 
-bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
-                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+namespace {
+
+// Everything an encoding depends on (a map is a pure function of these).
+struct TmapKey {
+  uint64_t base, dims[3], strides[2];
+  uint32_t box[3], rank, dtype, swz;
+  bool operator==(const TmapKey& o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
+};
+struct TmapSlot {
+  bool used = false;
+  TmapKey key;
+  CUtensorMap map;
+};
+constexpr int kTmapSlots = 512;
+std::mutex g_tmap_mu;
+TmapSlot g_tmap[kTmapSlots];
+
+bool encode_cached(CUtensorMap* map, const TmapKey& k) {
+  uint64_t h = 1469598103934665603ull;
+  const unsigned char* b = reinterpret_cast<const unsigned char*>(&k);
+  for (size_t i = 0; i < sizeof(k); ++i) h = (h ^ b[i]) * 1099511628211ull;
+  TmapSlot& slot = g_tmap[h % kTmapSlots];
+  {
+    std::lock_guard<std::mutex> lk(g_tmap_mu);
+    if (slot.used && slot.key == k) {
+      *map = slot.map;
+      return true;
+    }
+  }
   EncodeFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  for (uint32_t i = 0; i < k.rank; ++i) {
+    dims[i] = k.dims[i];
+    box[i] = k.box[i];
+    if (i + 1 < k.rank) strides[i] = k.strides[i];
+  }
   std::memset(map, 0, sizeof(*map));
-  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, (CUtensorMapDataType)k.dtype, k.rank, reinterpret_cast<void*>(k.base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)k.swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lk(g_tmap_mu);
+  slot.used = true;
+  slot.key = k;
+  slot.map = *map;
+  return true;
+}
+
+struct SmemSet {
+  const void* func;
+  int dev, bytes;
+};
+std::mutex g_smem_mu;
+SmemSet g_smem_set[256];
+int g_smem_n = 0;
+
+}  // namespace
+
+cudaError_t ensure_smem(const void* func, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  for (int i = 0; i < g_smem_n; ++i)
+    if (g_smem_set[i].func == func && g_smem_set[i].dev == dev && g_smem_set[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < g_smem_n; ++i)
+    if (g_smem_set[i].func == func && g_smem_set[i].dev == dev) {
+      g_smem_set[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (g_smem_n < 256) g_smem_set[g_smem_n++] = SmemSet{func, dev, bytes};
+  return cudaSuccess;
+}
+
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.base = reinterpret_cast<uint64_t>(base);
+  k.dims[0] = inner;
+  k.dims[1] = outer;
+  k.strides[0] = row_bytes;
+  k.box[0] = box_inner;
+  k.box[1] = box_outer;
+  k.rank = 2;
+  k.dtype = (uint32_t)dtype;
+  k.swz = (uint32_t)swz;
+  return encode_cached(map, k);
 }
 
 bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
                   uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2) {
-  EncodeFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {stride1, stride2};
-  const cuuint32_t box[3] = {b0, b1, b2};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  std::memset(map, 0, sizeof(*map));
-  return fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.base = reinterpret_cast<uint64_t>(base);
+  k.dims[0] = d0;
+  k.dims[1] = d1;
+  k.dims[2] = d2;
+  k.strides[0] = stride1;
+  k.strides[1] = stride2;
+  k.box[0] = b0;
+  k.box[1] = b1;
+  k.box[2] = b2;
+  k.rank = 3;
+  k.dtype = (uint32_t)dtype;
+  k.swz = (uint32_t)CU_TENSOR_MAP_SWIZZLE_NONE;
+  return encode_cached(map, k);
 }
 
 }  // namespace svdq

@@ -353,7 +353,7 @@ cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_
     b.x = a.x + (size_t)m0 * a.K;
     b.y = a.y + (size_t)m0 * a.N;
     const size_t smem = (size_t)AwqLayout(b.M, a.K).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(awq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(awq_kernel), (int)smem);
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: this grid may start while the previous
     // kernel in the stream finishes (see the kernel's wait before x)

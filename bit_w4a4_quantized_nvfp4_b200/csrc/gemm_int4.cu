@@ -509,7 +509,7 @@ cudaError_t launch_gemm_int4(const GemmArgs& a, cudaStream_t s) {
                           kScG, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(gemm_int4_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < a.num_sms ? tiles : a.num_sms;

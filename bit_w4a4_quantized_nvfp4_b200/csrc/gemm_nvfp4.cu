@@ -16,12 +16,12 @@
 //   warp 0      TMA producer (both CTAs): A/B code tiles (128B-swizzled,
 //               K-major) and UE4M3 scale atoms for its own rows; both CTAs'
 //               copies complete on the leader CTA's stage barrier. One extra
-//               stage per tile carries the P tile and the prepared L2 tile.
+//               stage opens each tile with the P tile and the prepared L2 tile.
 //   warp 1      TMEM allocator (both CTAs); in the leader CTA one thread
 //               issues, per 256-wide K stage, tcgen05.cp of the scale atoms
 //               (into both CTAs' tensor memory) and 4 x tcgen05.mma
-//               kind::mxf4nvf4 (K = 64); after the K loop, tcgen05.mma
-//               kind::f16 adds P (hi + lo) into the same accumulator.
+//               kind::mxf4nvf4 (K = 64); before the K loop, tcgen05.mma
+//               kind::f16 puts P (hi + lo) into the same accumulator.
 //   warps 2..9  epilogue (both CTAs), two warps per TMEM lane quadrant, each
 //               draining half of the 256 columns: tcgen05.ld, y = alpha*acc +
 //               bias (read through the L1 cache), convert, stage 32 x 64
@@ -127,6 +127,14 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // Programmatic dependent launch: the set-up above (barriers, tensor memory,
+  // tensor-map prefetch) may overlap the previous kernel in the stream; every
+  // input may be that kernel's output (the activation pass writes A, its
+  // scales and P) and y may still be read by it, so all global traffic comes
+  // after this wait. The next kernel may be scheduled at once: it waits for
+  // this one before it touches anything this one reads or writes.
+  if (threadIdx.x == 0) launch_dependents();
+  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -137,6 +145,20 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         const int tm = tile / p.tiles_n, tn = tile % p.tiles_n;
         const int row0 = tm * 256 + (int)rank * BM;      // this CTA's A rows
         const int col0 = tn * BN + (int)rank * (BN / 2);  // this CTA's B rows
+        if (has_lr) {
+          // the low-rank stage opens the tile, so its loads are hidden behind
+          // the K stages that follow it like any other stage's
+          const int s = it % kStages;
+          if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
+          uint8_t* st = sm.stage[s];
+          const uint32_t fb = mapa_shared(smem_u32(&sm.full[s]), 0);
+          const int pc = p.r / 8, lc = 2 * p.r / 8;  // 8-column groups
+          if (leader) mbar_expect_tx(&sm.full[s], 2u * (uint32_t)(pc + lc) * BM * 16);
+          // one copy each: [group][row][8 columns], the K-major core-matrix layout
+          tma_load_3d_pair(st, &tm_p, fb, 0, row0, 0);
+          tma_load_3d_pair(st + kABytes, &tm_l, fb, 0, col0, 0);
+          ++it;
+        }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
@@ -149,17 +171,6 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           tma_load_3d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfb, fb, 0, 4 * kb, 2 * tn);
         }
         if (!ok) break;
-        if (has_lr) {
-          const int s = it % kStages;
-          if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, p.wait_ns, p.err)) { ok = false; break; }
-          uint8_t* st = sm.stage[s];
-          const uint32_t fb = mapa_shared(smem_u32(&sm.full[s]), 0);
-          const int pc = p.r / 8, lc = 2 * p.r / 8;  // 8-column boxes
-          if (leader) mbar_expect_tx(&sm.full[s], 2u * (uint32_t)(pc + lc) * BM * 16);
-          for (int c = 0; c < pc; ++c) tma_load_2d_pair(st + c * BM * 16, &tm_p, fb, 8 * c, row0);
-          for (int c = 0; c < lc; ++c) tma_load_2d_pair(st + kABytes + c * BM * 16, &tm_l, fb, 8 * c, col0);
-          ++it;
-        }
       }
       if (!ok && leader) {
         // let the copies already issued by both CTAs land before the pair exits
@@ -186,6 +197,23 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           break;
         }
         tc_fence_after();
+        if (has_lr) {
+          // P (hi + lo) first: it opens the accumulator of the tile
+          const int s = it % kStages;
+          if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
+          const uint32_t st = smem_u32(sm.stage[s]);
+          const int half = p.r / 16;  // k16 steps per copy of P
+          for (int k = 0; k < 2 * half; ++k) {
+            const int kp = k % half;
+            const uint64_t ad = make_sdesc(st + 2 * kp * BM * 16, BM * 16, 128, kLayoutNone);
+            const uint64_t bd = make_sdesc(st + kABytes + 2 * k * BM * 16, BM * 16, 128, kLayoutNone);
+            if (elect_one()) mma_bf16_pair(acc, ad, bd, kIdescBf16, k > 0 ? 1u : 0u);
+            __syncwarp();
+          }
+          if (elect_one()) tc_commit_pair(&sm.empty[s], 0x3);
+          __syncwarp();
+          ++it;
+        }
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kStages;
           if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
@@ -213,28 +241,12 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               mma_nvfp4_pair(acc, da[j], db[j], kIdescNvfp4, tmem + kSfaCol + 4 * j, tmem + kSfbCol + 8 * j,
-                             (kb > 0 || j > 0) ? 1u : 0u);
+                             (has_lr || kb > 0 || j > 0) ? 1u : 0u);
             tc_commit_pair(&sm.empty[s], 0x3);
           }
           __syncwarp();
         }
         if (!ok) break;
-        if (has_lr) {
-          const int s = it % kStages;
-          if (!warp_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns, p.err)) { ok = false; break; }
-          const uint32_t st = smem_u32(sm.stage[s]);
-          const int half = p.r / 16;  // k16 steps per copy of P
-          for (int k = 0; k < 2 * half; ++k) {
-            const int kp = k % half;
-            const uint64_t ad = make_sdesc(st + 2 * kp * BM * 16, BM * 16, 128, kLayoutNone);
-            const uint64_t bd = make_sdesc(st + kABytes + 2 * k * BM * 16, BM * 16, 128, kLayoutNone);
-            if (elect_one()) mma_bf16_pair(acc, ad, bd, kIdescBf16, 1u);
-            __syncwarp();
-          }
-          if (elect_one()) tc_commit_pair(&sm.empty[s], 0x3);
-          __syncwarp();
-          ++it;
-        }
         if (elect_one()) tc_commit_pair(&sm.acc_full[i & 1], 0x3);
         __syncwarp();
       }
@@ -362,10 +374,13 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   ok = ok && make_tmap_3d(&tm_sfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.w_scales, 128, katoms, rb_w, 512, katoms * 512,
                           128, 4, 2);
   if (a.r > 0) {
-    ok = ok && make_tmap_2d(&tm_p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.P, a.r, a.M, (uint64_t)a.r * 2, 8, BM,
-                            CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && make_tmap_2d(&tm_l, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lr_up, 2 * a.r, a.N, (uint64_t)a.r * 4, 8,
-                            BN / 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+    // P [M, r] and lr_up [N, 2r] viewed as (8 columns, rows, column groups of 8):
+    // one box lands in shared memory as [group][row][8], the layout the
+    // kind::f16 MMA reads without swizzle
+    ok = ok && make_tmap_3d(&tm_p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.P, 8, a.M, (uint64_t)a.r / 8,
+                            (uint64_t)a.r * 2, 16, 8, BM, (uint32_t)a.r / 8);
+    ok = ok && make_tmap_3d(&tm_l, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.lr_up, 8, a.N, (uint64_t)a.r / 4,
+                            (uint64_t)a.r * 4, 16, 8, BN / 2, (uint32_t)a.r / 4);
   } else {
     tm_p = tm_a;
     tm_l = tm_a;
@@ -389,12 +404,23 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   p.wait_ns = a.wait_ns;
 
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(gemm_nvfp4_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
   const int pairs = a.num_sms / 2;
   const int grid = 2 * (tiles < pairs ? tiles : pairs);
-  gemm_nvfp4_kernel<<<grid, kThreads, smem, s>>>(tm_a, tm_b, tm_sfa, tm_sfb, tm_p, tm_l, tm_y, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, tm_a, tm_b, tm_sfa, tm_sfb, tm_p, tm_l, tm_y, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -86,8 +86,15 @@ cudaError_t launch_probe_wait(unsigned* err, unsigned long long limit_ns, cudaSt
 cudaError_t launch_probe_mma(int iters, int mode, int num_sms, unsigned* err, unsigned long long wait_ns,
                              cudaStream_t s);
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute is set once per (kernel, device, size): the
+// calls on the hot path then cost a table lookup.
+cudaError_t ensure_smem(const void* func, int bytes);
+
 // Host helper: encode a 2-D tiled tensor map (driver entry point looked up at
-// run time; no link-time dependency on libcuda).
+// run time; no link-time dependency on libcuda). Encodings are cached by
+// their full argument list, so a layer called again on the same buffers
+// reuses its maps.
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                   CUtensorMapSwizzle swz);

@@ -111,7 +111,7 @@ cudaError_t launch_probe_mma(int iters, int mode, int num_sms, unsigned* err, un
   // crossed over two SMs would each wait for the other's columns.
   const size_t smem = 120 * 1024;
   static_assert(kPStage + 1024 <= 120 * 1024, "one stage fits");
-  cudaError_t e = cudaFuncSetAttribute(probe_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(probe_mma_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   probe_mma_kernel<<<2 * (num_sms / 2), 128, smem, s>>>(iters, mode, err, wait_ns);
   return cudaGetLastError();

@@ -15,23 +15,30 @@
 // let every consumer warp run at its own pace, with no CTA-wide barrier
 // inside the K loop.
 //
-// Each of the 16 consumer warps owns one (row tile, K slice) block of 16 rows
-// x 64 columns in every other chunk (eight warps per chunk, two chunks in
-// work at a time). A lane holds 32 columns of one row: two NVFP4 groups,
-// whose independent dependency chains interleave, or half an INT4 group. The
-// warp quantises its block, writes x_hat back over its x block in the stage
-// and multiplies it by its K slice of the L1 tile on tensor cores (mma.sync
-// bf16, fp32 accumulate), so P needs no cross-warp exchange until the end,
-// where the eight partial sums of each row tile are added in a fixed order
-// and rounded to bf16 once.
+// Consumers: 8 warps cover one chunk, each a block of 16 rows x 64 columns
+// (row tile rt, K slice kp); the consumer warps form kPhases groups of 8 that
+// take chunks round-robin, so kPhases chunks are in work at once. Inside a
+// block a lane holds 16 columns (one NVFP4 group, a quarter of an INT4 group)
+// of two rows, p and p + 8: the two groups' dependency chains interleave, and
+// the lane's 16 inv_lambda values serve both rows. The warp writes x_hat back
+// over its x block in the stage and multiplies it by its K slice of the L1
+// tile on tensor cores (mma.sync bf16, fp32 accumulate), so P needs no
+// cross-warp exchange until the end, where the partial sums of each row tile
+// are added in a fixed order and rounded to bf16 once.
 //
-// Stage reuse: chunk c lives in stage c % S and the two warp groups take
-// alternate chunks, so S is kept even. A stage is then always refilled for
-// the group that released it, and no warp can wait on a full barrier more
-// than one phase ahead of it (with S odd, the previous user of a stage is
-// the other group, and a parity wait could pass on the wrong phase). The NVFP4 dequantisation step d = e4m3(s) * s_tx and
-// its reciprocal depend only on the 8-bit scale code, so each CTA tabulates
-// them once for all 256 codes.
+// Stage reuse: chunk c lives in stage c % S and the groups take chunks
+// round-robin, so S is a multiple of kPhases: a stage is then always refilled
+// for the group that released it, and no warp can wait on a full barrier more
+// than one phase ahead of it (otherwise a parity wait could pass on the wrong
+// phase). The NVFP4 dequantisation step d = e4m3(s) * s_tx and its reciprocal
+// depend only on the 8-bit scale code, so each CTA tabulates them once for
+// all 256 codes.
+//
+// Programmatic dependent launch: the kernel lets the next kernel in the
+// stream be scheduled at once (it waits for this one before it reads any
+// output), and reads or writes nothing that an earlier kernel may touch
+// (x, inv_lambda, the tensor scales, L1, the outputs) before
+// griddepcontrol.wait; only barrier set-up and L2 prefetches precede it.
 #include "device.cuh"
 #include "kernels.h"
 
@@ -42,9 +49,7 @@ constexpr int kRows = 32;                   // rows per CTA
 constexpr int kChunk = 256;                 // K columns per stage
 constexpr int kXBytes = kRows * kChunk * 2;
 constexpr int kXBoxBytes = kRows * 64 * 2;  // one [32 rows][64 cols] box, 128-byte swizzle
-constexpr int kConsumerWarps = 16;
-constexpr int kThreadsQA = (kConsumerWarps + 1) * 32;
-constexpr int kParts = 8;                   // partial P sums per row tile
+constexpr int kKParts = kChunk / 64;        // 64-column K slices per chunk
 constexpr int kSmemLimit = 232448;          // dynamic shared memory per CTA on sm_100
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -80,18 +85,71 @@ __device__ __forceinline__ void mul2(float a0, float a1, float b0, float b1, flo
   asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(D));
 }
 
-// smooth 8 bf16 values (one 16-byte word of x) by their inv_lambda: returns
-// bf16x2 words of x_hat and folds |x_hat| into `amax2`
-__device__ __forceinline__ void smooth8(const uint4 xv, const float* il, uint32_t (&hb)[4],
-                                        __nv_bfloat162& amax2) {
-  const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+// per half: |max(|a|, |b|)| in magnitude (the sign bits are garbage and are
+// cleared by the caller); one instruction for abs + max of a bf16 pair
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// per 16-bit half: unsigned maximum
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// element i of four float4
+__device__ __forceinline__ float f4at(const float4 (&v)[4], int i) {
+  const float4 q = v[i >> 2];
+  return (i & 3) == 0 ? q.x : (i & 3) == 1 ? q.y : (i & 3) == 2 ? q.z : q.w;
+}
+
+// smooth 16 bf16 values (two 16-byte words of x) by their inv_lambda: x_hat
+// as 8 bf16x2 words, and the running |x_hat| maximum of the 16 (in both halves)
+__device__ __forceinline__ uint32_t smooth16(const uint4 xa, const uint4 xb, const float4 (&il)[4],
+                                             uint32_t (&hb)[8]) {
+  const uint32_t w[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+  uint32_t am = 0;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < 8; ++j) {
     float p0, p1;
-    mul2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u), il[2 * j], il[2 * j + 1], p0, p1);
+    mul2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u), f4at(il, 2 * j), f4at(il, 2 * j + 1),
+         p0, p1);
     hb[j] = pack_bf16x2(p0, p1);
-    amax2 = __hmax2(amax2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&hb[j])));
+    am = absmax_bf16x2(am, hb[j]);
   }
+  return am & 0x7FFF7FFFu;
+}
+
+// 16 NVFP4 codes of a group: E2M1 of fl(x_hat * rcp) for the 8 x_hat words
+// (element 2j of the group in the low nibble of byte j)
+__device__ __forceinline__ uint2 e2m1_group(const uint32_t (&hb)[8], float rcp) {
+  float q[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    mul2(__uint_as_float(hb[j] << 16), __uint_as_float(hb[j] & 0xFFFF0000u), rcp, rcp, q[2 * j], q[2 * j + 1]);
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w[h])
+        : "f"(q[8 * h]), "f"(q[8 * h + 1]), "f"(q[8 * h + 2]), "f"(q[8 * h + 3]), "f"(q[8 * h + 4]),
+          "f"(q[8 * h + 5]), "f"(q[8 * h + 6]), "f"(q[8 * h + 7]));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// bf16 bits of the larger of the two (non-negative) halves
+__device__ __forceinline__ uint32_t max_half(uint32_t am) {
+  const uint32_t lo = am & 0xFFFFu, hi = am >> 16;
+  return lo > hi ? lo : hi;
 }
 
 __device__ __forceinline__ void named_sync(int id, int threads) {
@@ -101,36 +159,39 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
 template <int PREC, int NT>
 struct Cfg {
   static constexpr int kR = NT * 8;
-  static constexpr int KW = 64;                                 // columns per warp block
-  static constexpr int kKParts = kChunk / KW;                   // K slices per chunk
-  static constexpr int kPhases = kConsumerWarps / 2 / kKParts;  // chunks in work per CTA
-  static constexpr int kConsumers = kConsumerWarps / kPhases;   // warps reading one chunk
+  static constexpr int kConsumerWarps = NT > 4 ? 16 : 24;      // registers: 16 warps when P holds 6-8 tiles
+  static constexpr int kPhases = kConsumerWarps / 8;           // chunks in work per CTA
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  // registers per thread: the most that fits in the 64K-entry register file
+  // when the CTA's warps are counted in groups of four (8-register steps)
+  static constexpr int kMaxRegs = ((65536 / ((kConsumerWarps + 1 + 3) / 4 * 4 * 32)) / 8) * 8;
+  static constexpr int kParts = kPhases * kKParts;             // partial P sums per row tile
   static constexpr int kL1Bytes = NT ? kChunk * kR * 2 : 0;
   static constexpr int kIlBytes = kChunk * 4;
   static constexpr int kStageBytes = ((kXBytes + kL1Bytes + kIlBytes + 1023) / 1024) * 1024;
   static constexpr int kFixed = 1024 + 256 * 8 + 256;
   static constexpr int kFit = (kSmemLimit - kFixed) / kStageBytes;
-  static constexpr int kStages = ((kFit > 8 ? 8 : kFit) / kPhases) * kPhases;
+  static constexpr int kStages = ((kFit > 9 ? 9 : kFit) / kPhases) * kPhases;
   static constexpr size_t kSmem = (size_t)kFixed + (size_t)kStages * kStageBytes;
   // the L1 tile rows are 2r bytes; the TMA swizzle span equals the row (32/64/128 B)
   static constexpr uint32_t kSwzMask = kR <= 16 ? 1u : (kR == 32 ? 3u : 7u);
-  static_assert(kKParts * kPhases == kParts, "eight partial sums per row tile");
   static_assert((size_t)kParts * kRows * (kR > 0 ? kR : 1) * 4 <= (size_t)kStages * kStageBytes,
                 "the reduction buffer fits in the stages");
   static_assert(2 * kStages * 8 + 4 <= 256, "barriers fit their reserve");
-  static_assert(kStages >= 2 && kStages % kPhases == 0, "a stage is reused by one warp group only");
+  static_assert(kStages >= kPhases && kStages % kPhases == 0, "a stage is reused by one warp group only");
 };
 
 // PREC 0 = NVFP4 (group 16, E4M3 scales in the tiled layout), 1 = INT4
 // (group 64, bf16 scales row-major, row pitch int4_act_scale_pitch). NT = r / 8
 // tiles of the P output.
 template <int PREC, int NT>
-__global__ void __launch_bounds__(kThreadsQA, 1)
+__global__ void __maxnreg__((Cfg<PREC, NT>::kMaxRegs))
 quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
                  QuantActArgs a, unsigned* err, unsigned long long wait_ns) {
   using C = Cfg<PREC, NT>;
   constexpr int kR = C::kR;
   constexpr int S = C::kStages;
+  constexpr int CW = C::kConsumerWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = base;                                       // S x kStageBytes
@@ -148,14 +209,24 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   const int M = a.M, K = a.K;
   const int nchunks = (K + kChunk - 1) / kChunk;
 
+  if (threadIdx.x == 0) launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::kConsumers);
+      mbar_init(&empty[s], 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == CW && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    if (NT) tma_prefetch_desc(&tm_l1);
+    for (int c = 0; c < nchunks && c < S; ++c)
+      for (int b = 0; b < min(kChunk, K - c * kChunk) / 64; ++b) tma_prefetch_l2_2d(&tm_x, c * kChunk + 64 * b, row0);
+  }
+  // every input may be the previous kernel's output, every output may still
+  // be read by it
+  grid_dependency_wait();
   const float s_tx = PREC == 0 ? a.tensor_scale[1] : 1.0f;
   if (PREC == 0 && threadIdx.x < 256) {
     const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), s_tx);
@@ -163,11 +234,9 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
+  if (warp == CW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_x);
-      if (NT) tma_prefetch_desc(&tm_l1);
       int c = 0;
       bool ok = true;
       for (; c < nchunks; ++c) {
@@ -193,23 +262,39 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   }
 
   // -------------------------------------------------------------- consumers
-  const int rt = warp & 1;                     // row tile
-  const int kp = (warp >> 1) % C::kKParts;     // K slice within a chunk
-  const int phase = (warp >> 1) / C::kKParts;  // chunk phase
-  const int rl = lane & 15, h = lane >> 4;
-  const int lr = rt * 16 + rl;                 // local row
-  const int m = row0 + lr;
-  const bool row_ok = m < M;
+  const int rt = warp & 1;                 // row tile
+  const int kp = (warp >> 1) & 3;          // K slice within a chunk
+  const int phase = warp >> 3;             // chunk phase
+  const int p = lane & 7, cq = lane >> 3;  // rows p and p + 8 of the tile, columns 16 cq .. 16 cq + 15
+  const int lr0 = rt * 16 + p;             // local rows lr0, lr0 + 8
+  const int m0 = row0 + lr0, m1 = m0 + 8;
+  const bool ok0 = m0 < M, ok1 = m1 < M;
   const float six_t = __fmul_rn(6.0f, s_tx);
-  // this lane's outputs, advanced by one chunk per step: codes of columns
-  // c*256 + kp*64 + 32h .. +31, and the scale word (NVFP4: the 4 scales of
-  // 64-column atom 4c + kp in row m; INT4: scale 4c + kp of row m)
-  const int m_c = row_ok ? m : 0;
-  uint8_t* code_ptr = a.codes + (size_t)m_c * (K / 2) + kp * 32 + h * 16;
-  uint8_t* scale_ptr =
-      PREC == 0 ? static_cast<uint8_t*>(a.scales) + ((size_t)(m_c / 128) * (K / 64) + kp) * 512 + 16 * (m_c % 32) +
-                      4 * ((m_c % 128) / 32)
-                : static_cast<uint8_t*>(a.scales) + ((size_t)m_c * int4_act_scale_pitch(K) + kp) * 2;
+  // this lane's x words in a block: 16-byte units 2cq, 2cq + 1 of rows p, p + 8
+  // (128-byte swizzle: unit u of row r sits at (u ^ (r & 7)) << 4)
+  const uint32_t xoff0 = (uint32_t)(kp * kXBoxBytes + lr0 * 128 + (((2 * cq) ^ p) << 4));
+  const uint32_t xoff1 = (uint32_t)(kp * kXBoxBytes + lr0 * 128 + (((2 * cq + 1) ^ p) << 4));
+  const uint32_t iloff = (uint32_t)(kXBytes + C::kL1Bytes + (kp * 64 + 16 * cq) * 4);
+  // outputs, advanced by one chunk per step
+  uint8_t* code0 = a.codes + (size_t)(ok0 ? m0 : 0) * (K / 2) + kp * 32 + cq * 8;
+  uint8_t* code1 = a.codes + (size_t)(ok1 ? m1 : 0) * (K / 2) + kp * 32 + cq * 8;
+  uint8_t* sc0;
+  uint8_t* sc1;
+  if constexpr (PREC == 0) {
+    auto at = [&](int m) {
+      return static_cast<uint8_t*>(a.scales) + ((size_t)(m / 128) * (K / 64) + kp) * 512 + 16 * (m % 32) +
+             4 * ((m % 128) / 32) + cq;
+    };
+    sc0 = at(ok0 ? m0 : 0);
+    sc1 = at(ok1 ? m1 : 0);
+  } else {
+    sc0 = static_cast<uint8_t*>(a.scales) + ((size_t)(ok0 ? m0 : 0) * int4_act_scale_pitch(K) + kp) * 2;
+    sc1 = static_cast<uint8_t*>(a.scales) + ((size_t)(ok1 ? m1 : 0) * int4_act_scale_pitch(K) + kp) * 2;
+  }
+  // P fragments: A from this warp's x_hat block, B from rows kp*64 .. of the L1 tile
+  const int ar = lane & 15;
+  const uint32_t aoff = (uint32_t)(kp * kXBoxBytes + (rt * 16 + ar) * 128);
+  const int ab = lane >> 4;
 
   float acc[NT > 0 ? NT : 1][4];
 #pragma unroll
@@ -218,103 +303,96 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   bool ok = true;
   for (int c = phase; c < nchunks; c += C::kPhases) {
     const int s = c % S;
-    const uint8_t* st = stages + s * C::kStageBytes;
+    uint8_t* st = stages + s * C::kStageBytes;
     if (!warp_wait(&full[s], (c / S) & 1, wait_ns, err)) {
       ok = false;
       break;
     }
     const int kcols = min(kChunk, K - c * kChunk);
-    if (kp * C::KW < kcols) {  // warp-uniform: the block lies inside K
-      const int cc = kp * C::KW + h * (C::KW / 2);  // first chunk column of this lane
-      // this warp's x block: rows 16rt .. of box kp (128-byte lines, units swizzled by line)
-      uint8_t* xblk = stages + s * C::kStageBytes + kp * kXBoxBytes + rt * 16 * 128;
-      const uint8_t* xrow = xblk + rl * 128;
-      const float* ils = reinterpret_cast<const float*>(st + kXBytes + C::kL1Bytes) + cc;
-      // smooth 32 columns: x_hat words hb[0..15], |x_hat| maxima of the two 16-column halves
-      uint32_t hb[16];
-      __nv_bfloat162 amax2[2] = {__float2bfloat162_rn(0.f), __float2bfloat162_rn(0.f)};
+    if (kp * 64 < kcols) {  // warp-uniform: the block lies inside K
+      const uint4 xa0 = *reinterpret_cast<const uint4*>(st + xoff0);
+      const uint4 xb0 = *reinterpret_cast<const uint4*>(st + xoff1);
+      const uint4 xa1 = *reinterpret_cast<const uint4*>(st + xoff0 + 8 * 128);
+      const uint4 xb1 = *reinterpret_cast<const uint4*>(st + xoff1 + 8 * 128);
+      float4 il[4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(xrow + (((4 * h + v) ^ (lr & 7)) << 4));
-        float il[8];
-        *reinterpret_cast<float4*>(il) = *reinterpret_cast<const float4*>(ils + 8 * v);
-        *reinterpret_cast<float4*>(il + 4) = *reinterpret_cast<const float4*>(ils + 8 * v + 4);
-        uint32_t hv[4];
-        smooth8(xv, il, hv, amax2[v >> 1]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) hb[4 * v + j] = hv[j];
-      }
+      for (int v = 0; v < 4; ++v) il[v] = *reinterpret_cast<const float4*>(st + iloff + 16 * v);
+      uint32_t hb0[8], hb1[8];
+      const uint32_t am0 = smooth16(xa0, xb0, il, hb0);
+      const uint32_t am1 = smooth16(xa1, xb1, il, hb1);
       // x_hat over the lane's own x words, for the P product
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        *reinterpret_cast<uint4*>(xblk + rl * 128 + (((4 * h + v) ^ (lr & 7)) << 4)) =
-            make_uint4(hb[4 * v], hb[4 * v + 1], hb[4 * v + 2], hb[4 * v + 3]);
+      *reinterpret_cast<uint4*>(st + xoff0) = make_uint4(hb0[0], hb0[1], hb0[2], hb0[3]);
+      *reinterpret_cast<uint4*>(st + xoff1) = make_uint4(hb0[4], hb0[5], hb0[6], hb0[7]);
+      *reinterpret_cast<uint4*>(st + xoff0 + 8 * 128) = make_uint4(hb1[0], hb1[1], hb1[2], hb1[3]);
+      *reinterpret_cast<uint4*>(st + xoff1 + 8 * 128) = make_uint4(hb1[4], hb1[5], hb1[6], hb1[7]);
       const size_t cstep = (size_t)c;
 
       if constexpr (PREC == 0) {
-        // two NVFP4 groups of 16 per lane
-        uint32_t code[4], sfw = 0;
-#pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-          const float amax = fmaxf(__low2float(amax2[gi]), __high2float(amax2[gi]));
-          const uint32_t sf = cvt_e4m3(__fdiv_rn(amax, six_t)) & 0xFFu;
-          const float2 rt_e = rtab[sf];
-          float q[16];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            mul2(__uint_as_float(hb[8 * gi + j] << 16), __uint_as_float(hb[8 * gi + j] & 0xFFFF0000u), rt_e.x,
-                 rt_e.x, q[2 * j], q[2 * j + 1]);
-          // a zero dequantisation step codes the whole group as +0
-          const bool zero = rt_e.y != 0.f;
-          code[2 * gi] = zero ? 0u : cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q));
-          code[2 * gi + 1] = zero ? 0u : cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(q + 8));
-          sfw |= sf << (8 * gi);
+        // one NVFP4 group of 16 per row
+        const uint32_t sf0 = cvt_e4m3(__fdiv_rn(__uint_as_float(max_half(am0) << 16), six_t));
+        const uint32_t sf1 = cvt_e4m3(__fdiv_rn(__uint_as_float(max_half(am1) << 16), six_t));
+        const float2 r0 = rtab[sf0], r1 = rtab[sf1];
+        uint2 c0 = e2m1_group(hb0, r0.x);
+        uint2 c1 = e2m1_group(hb1, r1.x);
+        // a zero dequantisation step codes the whole group as +0
+        if (r0.y != 0.f) c0 = make_uint2(0u, 0u);
+        if (r1.y != 0.f) c1 = make_uint2(0u, 0u);
+        if (ok0) {
+          *reinterpret_cast<uint2*>(code0 + cstep * 128) = c0;
+          sc0[cstep * 4 * 512] = (uint8_t)sf0;
         }
-        // the row's four scales of this 64-column atom: lanes h = 0 and 1
-        const uint32_t sfw_hi = __shfl_xor_sync(0xffffffffu, sfw, 16);
-        if (row_ok) {
-          *reinterpret_cast<uint4*>(code_ptr + cstep * 128) = make_uint4(code[0], code[1], code[2], code[3]);
-          if (h == 0) *reinterpret_cast<uint32_t*>(scale_ptr + cstep * 4 * 512) = sfw | (sfw_hi << 16);
+        if (ok1) {
+          *reinterpret_cast<uint2*>(code1 + cstep * 128) = c1;
+          sc1[cstep * 4 * 512] = (uint8_t)sf1;
         }
       } else {
-        // half an INT4 group of 64 per lane
-        __nv_bfloat162 am = __hmax2(amax2[0], amax2[1]);
-        float amax = fmaxf(__low2float(am), __high2float(am));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-        const uint32_t sb = f32_to_bf16_bits(__fdiv_rn(amax, 7.0f));
-        const float sfv = bf16_bits_to_f32(sb);
-        uint32_t code[4] = {0u, 0u, 0u, 0u};
-        if (sfv != 0.f) {
-          const float inv = __frcp_rn(sfv);
+        // a quarter of an INT4 group of 64 per row: the group maximum over the
+        // four lanes cq = 0..3 of each row (both rows in one word: bf16 bits of
+        // non-negative values order like unsigned integers)
+        uint32_t am = max_half(am0) | (max_half(am1) << 16);
+        am = max_u16x2(am, __shfl_xor_sync(0xffffffffu, am, 8));
+        am = max_u16x2(am, __shfl_xor_sync(0xffffffffu, am, 16));
+        const uint32_t sb0 = f32_to_bf16_bits(__fdiv_rn(__uint_as_float(am << 16), 7.0f));
+        const uint32_t sb1 = f32_to_bf16_bits(__fdiv_rn(__uint_as_float(am & 0xFFFF0000u), 7.0f));
+        auto quant = [&](const uint32_t (&hb)[8], uint32_t sb) {
+          const float sfv = bf16_bits_to_f32(sb);
+          uint2 code = make_uint2(0u, 0u);
+          if (sfv != 0.f) {
+            const float inv = __frcp_rn(sfv);
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 8; ++j) {
               float q0, q1;
-              const uint32_t hw = hb[4 * w + j];
-              mul2(__uint_as_float(hw << 16), __uint_as_float(hw & 0xFFFF0000u), inv, inv, q0, q1);
+              mul2(__uint_as_float(hb[j] << 16), __uint_as_float(hb[j] & 0xFFFF0000u), inv, inv, q0, q1);
               const int i0 = max(-8, min(7, __float2int_rn(q0)));
               const int i1 = max(-8, min(7, __float2int_rn(q1)));
-              code[w] |= (((uint32_t)i0 & 0xFu) | (((uint32_t)i1 & 0xFu) << 4)) << (8 * j);
+              const uint32_t byte = ((uint32_t)i0 & 0xFu) | (((uint32_t)i1 & 0xFu) << 4);
+              if (j < 4) code.x |= byte << (8 * j);
+              else code.y |= byte << (8 * (j - 4));
             }
           }
+          return code;
+        };
+        const uint2 c0 = quant(hb0, sb0), c1 = quant(hb1, sb1);
+        if (ok0) {
+          *reinterpret_cast<uint2*>(code0 + cstep * 128) = c0;
+          if (cq == 0) *reinterpret_cast<uint16_t*>(sc0 + cstep * 8) = (uint16_t)sb0;
         }
-        if (row_ok) {
-          *reinterpret_cast<uint4*>(code_ptr + cstep * 128) = make_uint4(code[0], code[1], code[2], code[3]);
-          if (h == 0) *reinterpret_cast<uint16_t*>(scale_ptr + cstep * 8) = (uint16_t)sb;
+        if (ok1) {
+          *reinterpret_cast<uint2*>(code1 + cstep * 128) = c1;
+          if (cq == 0) *reinterpret_cast<uint16_t*>(sc1 + cstep * 8) = (uint16_t)sb1;
         }
       }
 
       if constexpr (NT > 0) {
         __syncwarp();
-        // this block's share of P: x_hat[16 x KW] times rows kp*KW .. of the L1 tile
-        const uint32_t l1base = smem_u32(st + kXBytes);
+        // this block's share of P: x_hat[16 x 64] times rows kp*64 .. of the L1 tile
+        const uint32_t sb = smem_u32(st);
+        const uint32_t l1base = sb + kXBytes;
 #pragma unroll
-        for (int ks = 0; ks < C::KW / 16; ++ks) {
+        for (int ks = 0; ks < 4; ++ks) {
           uint32_t a0, a1, a2, a3;
-          const int ar = lane & 15, au = 2 * ks + (lane >> 4);
-          ldsm_x4(smem_u32(xblk) + ar * 128 + ((au ^ (ar & 7)) << 4), a0, a1, a2, a3);
-          const int k0 = kp * C::KW + ks * 16;
+          ldsm_x4(sb + aoff + (((2 * ks + ab) ^ (ar & 7)) << 4), a0, a1, a2, a3);
+          const int k0 = kp * 64 + ks * 16;
 #pragma unroll
           for (int t = 0; t < NT; t += 2) {
             uint32_t b0, b1, b2, b3;
@@ -342,31 +420,29 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   }
 
   if (!ok && lane == 0) *abort_flag = 1;
-  named_sync(1, kConsumerWarps * 32);
+  named_sync(1, CW * 32);
   // after a timed-out stage, copies may still be landing in the stages: write
   // nothing more
   if (*abort_flag) return;
   if constexpr (NT > 0) {
-    // fixed-order reduction of the eight K parts, then one bf16 rounding
-    const int part = phase * C::kKParts + kp;
+    // fixed-order reduction of the partial sums, then one bf16 rounding
+    const int part = phase * kKParts + kp;
     const int g = lane >> 2, t4 = lane & 3;
     float* rb = red + (size_t)part * kRows * kR;
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       const int j = t * 8 + 2 * t4;
-      rb[(rt * 16 + g) * kR + j] = acc[t][0];
-      rb[(rt * 16 + g) * kR + j + 1] = acc[t][1];
-      rb[(rt * 16 + g + 8) * kR + j] = acc[t][2];
-      rb[(rt * 16 + g + 8) * kR + j + 1] = acc[t][3];
+      *reinterpret_cast<float2*>(rb + (rt * 16 + g) * kR + j) = make_float2(acc[t][0], acc[t][1]);
+      *reinterpret_cast<float2*>(rb + (rt * 16 + g + 8) * kR + j) = make_float2(acc[t][2], acc[t][3]);
     }
-    named_sync(1, kConsumerWarps * 32);
-    for (int e = threadIdx.x; e < kRows * kR; e += kConsumerWarps * 32) {
+    named_sync(1, CW * 32);
+    for (int e = threadIdx.x; e < kRows * kR; e += CW * 32) {
       const int er = e / kR, j = e % kR;
       const int mm = row0 + er;
       if (mm >= M) continue;
       float v = red[e];
 #pragma unroll
-      for (int p = 1; p < kParts; ++p) v += red[p * kRows * kR + e];
+      for (int q = 1; q < C::kParts; ++q) v += red[q * kRows * kR + e];
       a.P[(size_t)mm * kR + j] = (uint16_t)f32_to_bf16_bits(v);
     }
   }
@@ -389,10 +465,20 @@ cudaError_t launch_t(const QuantActArgs& a, unsigned* err, unsigned long long wa
     tm_l1 = tm_x;
   }
   auto k = quant_act_kernel<PREC, NT>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(k), (int)C::kSmem);
   if (e != cudaSuccess) return e;
-  const int grid = (a.M + kRows - 1) / kRows;
-  k<<<grid, kThreadsQA, C::kSmem, s>>>(tm_x, tm_l1, a, err, wait_ns);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.M + kRows - 1) / kRows);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, tm_x, tm_l1, a, err, wait_ns);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

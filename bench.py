@@ -316,6 +316,8 @@ def run_cuda(args):
         out["clocks"] = clk
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(d, rows=args.cpu_rows)
+    if rank == 0 and not args.no_qkv:
+        out["qkv_epilogue"] = bench_qkv(svdq, pw, L1, b, x, qa, flush, M, N, K)
     if rank == 0 and not args.no_awq:
         out["awq_gemv"] = [bench_awq(svdq, P, m) for m in synth.CONFIGS["c2_awq_gemv"]["Ms"]]
     if rank == 0 and not args.no_int4:
@@ -401,6 +403,48 @@ def e2e_pipelined(svdq, pw, L1, b, xh, M, N, K, steps, world):
     ms = run(steps)
     barrier(world)
     return ms
+
+
+def bench_qkv(svdq, pw, L1, b, x, qa, flush, M, N, K, steps=30):
+    """The workload as the grouped Q/K/V projection of a DiT block (24 heads
+    of 128 per section) followed by per-head RMSNorm of Q and K and the rotary
+    embedding: fused into the GEMM's epilogue (svdq_w4a4_linear_qkv) against
+    the plain layer followed by the separate pass (svdq_qkv_norm_rope). One
+    step = activation pass + GEMM (+ pass), L2 flushed before each step,
+    medians of CUDA-event times."""
+    heads = N // 384
+    e = synth.qkv_epilogue_inputs(synth.CONFIGS[WORKLOAD]["seed"], M, 128, heads)
+    wq, wk = bf16_dev(e["wq"]), bf16_dev(e["wk"])
+    cos, sin = torch.from_numpy(e["cos"]).cuda(), torch.from_numpy(e["sin"]).cuda()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+
+    def fused():
+        svdq.quantize_act(x, pw, L1, out=qa)
+        svdq.w4a4_linear_qkv(qa, pw, heads, wq, wk, e["eps"], cos, sin, b, out=y)
+
+    def unfused():
+        svdq.quantize_act(x, pw, L1, out=qa)
+        svdq.w4a4_linear(qa, pw, b, out=y)
+        svdq.qkv_norm_rope(y, heads, wq, wk, e["eps"], cos, sin)
+
+    res = {}
+    for name, fn in (("fused_ms", fused), ("unfused_ms", unfused)):
+        ts = []
+        for i in range(steps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        res[name] = round(statistics.median(ts), 5)
+    svdq.device_error()
+    res["speedup"] = round(res["unfused_ms"] / res["fused_ms"], 4)
+    res["workload"] = (f"fused-QKV projection M{M} K{K} N{N} ({heads} heads of 128 per section) + RMSNorm of Q, K "
+                       "+ rotary embedding")
+    return res
 
 
 def bench_int4(svdq, P, steps=10):
@@ -597,6 +641,7 @@ def main():
     ap.add_argument("--no-awq", action="store_true")
     ap.add_argument("--no-int4", action="store_true")
     ap.add_argument("--no-probe", action="store_true")
+    ap.add_argument("--no-qkv", action="store_true")
     ap.add_argument("--oracle-configs", action="store_true",
                     help="only time the CPU oracle on every workload (no GPU needed) and exit")
     args = ap.parse_args()

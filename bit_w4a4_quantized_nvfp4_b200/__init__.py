@@ -28,7 +28,7 @@ import torch
 __all__ = [
     "NVFP4", "INT4", "Status", "SvdqError", "PackedWeight", "QuantAct", "AwqWeight",
     "library_path", "load", "scale_bytes", "pack_weight", "quantize_act", "w4a4_linear",
-    "svdq_linear", "awq_pack_weight", "awq_w4a16_linear", "device_error", "set_wait_limit_ns",
+    "w4a4_linear_qkv", "qkv_norm_rope", "svdq_linear", "awq_pack_weight", "awq_w4a16_linear", "device_error", "set_wait_limit_ns",
     "probe_convert", "probe_wait_timeout", "probe_mma_peak", "debug_force_arch",
 ]
 
@@ -69,6 +69,8 @@ SIGNATURES = {
     "svdq_pack_weight": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P]),
     "svdq_quantize_act": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
+    "svdq_w4a4_linear_qkv": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P]),
+    "svdq_qkv_norm_rope": (_I, [_I, _I, _P, _P, _F, _P, _P, _P, _P]),
     "awq_pack_weight": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "awq_w4a16_linear": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_device_error": (_I, [_P]),
@@ -292,6 +294,56 @@ def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = N
     _check("svdq_w4a4_linear", load().svdq_w4a4_linear(pw.prec, M, K, N, pw.r, *ptrs, _OUT[out_dtype],
                                                        _stream(stream)))
     return out
+
+
+def w4a4_linear_qkv(qa: QuantAct, pw: PackedWeight, heads: int, norm_q: torch.Tensor, norm_k: torch.Tensor,
+                    eps: float, cos: torch.Tensor, sin: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                    stream=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """svdq_w4a4_linear_qkv: the NVFP4 layer as a grouped Q/K/V projection (N =
+    3 * heads * 128) with per-head RMSNorm of Q and K and the rotary embedding
+    in the GEMM's epilogue. cos, sin: fp32 [M, 64]."""
+    M, K, N = qa.M, qa.K, pw.N
+    _check_packed(pw)
+    _need(pw.prec == NVFP4 and qa.prec == NVFP4, "the fused QKV epilogue is NVFP4 only")
+    _need(qa.K == pw.K and qa.r == pw.r, "activations (K {}, r {}) do not match the weight (K {}, r {})",
+          qa.K, qa.r, pw.K, pw.r)
+    _need(heads > 0 and N == 3 * heads * 128, "N = {} is not 3 * heads * 128 with heads = {}", N, heads)
+    _is(qa.codes, torch.uint8, (M, K // 2), "qa.codes")
+    _at_least(qa.scales, torch.uint8, scale_bytes(qa.prec, M, K), "qa.scales")
+    if qa.r:
+        _is(qa.P, torch.bfloat16, (M, qa.r), "qa.P")
+    _is(norm_q, torch.bfloat16, (128,), "norm_q")
+    _is(norm_k, torch.bfloat16, (128,), "norm_k")
+    _is(cos, torch.float32, (M, 64), "cos")
+    _is(sin, torch.float32, (M, 64), "sin")
+    if bias is not None:
+        _is(bias, torch.bfloat16, (N,), "bias")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.codes.device)
+    else:
+        _is(out, torch.bfloat16, (M, N), "out")
+    ptrs = _ptrs(qa.codes, qa.scales, qa.P, pw.codes, pw.scales, pw.tensor_scale, pw.lr_up, bias, norm_q, norm_k)
+    pc, ps, po = _ptrs(cos, sin, out)
+    _check("svdq_w4a4_linear_qkv", load().svdq_w4a4_linear_qkv(M, K, heads, pw.r, *ptrs, float(eps), pc, ps, po,
+                                                               _stream(stream)))
+    return out
+
+
+def qkv_norm_rope(y: torch.Tensor, heads: int, norm_q: torch.Tensor, norm_k: torch.Tensor, eps: float,
+                  cos: torch.Tensor, sin: torch.Tensor, stream=None) -> torch.Tensor:
+    """svdq_qkv_norm_rope: per-head RMSNorm + rotary embedding of the Q and K
+    sections of a bf16 grouped-QKV output y [M, 3 * heads * 128], in place."""
+    _need(y.dim() == 2 and y.dtype == torch.bfloat16, "y: expected bfloat16 [M, N]")
+    M, N = y.shape
+    _need(heads > 0 and N == 3 * heads * 128, "N = {} is not 3 * heads * 128 with heads = {}", N, heads)
+    _is(norm_q, torch.bfloat16, (128,), "norm_q")
+    _is(norm_k, torch.bfloat16, (128,), "norm_k")
+    _is(cos, torch.float32, (M, 64), "cos")
+    _is(sin, torch.float32, (M, 64), "sin")
+    pq, pk, pc, ps, py = _ptrs(norm_q, norm_k, cos, sin, y)
+    _check("svdq_qkv_norm_rope", load().svdq_qkv_norm_rope(M, heads, pq, pk, float(eps), pc, ps, py,
+                                                           _stream(stream)))
+    return y
 
 
 def svdq_linear(x: torch.Tensor, pw: PackedWeight, L1: Optional[torch.Tensor],

@@ -301,6 +301,54 @@ svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const
   return from_cuda(p == SVDQ_NVFP4 ? launch_gemm_nvfp4(a, s) : launch_gemm_int4(a, s));
 }
 
+svdq_status svdq_w4a4_linear_qkv(int M, int K, int heads, int r, const uint8_t* x_codes, const void* x_scales,
+                                 const uint16_t* P, const uint8_t* w_codes, const void* w_scales,
+                                 const float* w_tensor_scale, const uint16_t* lr_up, const uint16_t* bias,
+                                 const uint16_t* norm_q, const uint16_t* norm_k, float eps, const float* cos_t,
+                                 const float* sin_t, uint16_t* y, void* stream) {
+  svdq_status st = check_common(SVDQ_NVFP4, K, r);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || heads <= 0 || heads > (1 << 20) / 384) return SVDQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f && eps < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!x_codes || !x_scales || !w_codes || !w_scales || !w_tensor_scale || !y || !norm_q || !norm_k || !cos_t ||
+      !sin_t)
+    return SVDQ_ERR_INVALID_ARG;
+  if (r > 0 && (!P || !lr_up)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(w_tensor_scale) || !aligned16(y) || !aligned16(norm_q) || !aligned16(norm_k) ||
+      !aligned16(cos_t) || !aligned16(sin_t) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3)) ||
+      (r > 0 && (!aligned16(P) || !aligned16(lr_up))))
+    return SVDQ_ERR_ALIGN;
+  unsigned* err = nullptr;
+  int sms = 0;
+  if ((st = device_info(&err, &sms)) != SVDQ_OK) return st;
+  const int N = 3 * heads * 128;
+  GemmArgs a{x_codes, x_scales, P,  w_codes, w_scales, w_tensor_scale, lr_up, bias, y, M, K, N, r, (int)SVDQ_OUT_BF16,
+             err, g_wait_ns.load(), sms};
+  a.qkv_heads = heads;
+  a.norm_q = norm_q;
+  a.norm_k = norm_k;
+  a.eps = eps;
+  a.cos_t = cos_t;
+  a.sin_t = sin_t;
+  return from_cuda(launch_gemm_nvfp4(a, static_cast<cudaStream_t>(stream)));
+}
+
+svdq_status svdq_qkv_norm_rope(int M, int heads, const uint16_t* norm_q, const uint16_t* norm_k, float eps,
+                               const float* cos_t, const float* sin_t, uint16_t* y, void* stream) {
+  if (M < 0 || heads <= 0 || heads > (1 << 20) / 384) return SVDQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f && eps < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!norm_q || !norm_k || !cos_t || !sin_t || !y) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(norm_q) || !aligned16(norm_k) || !aligned16(cos_t) || !aligned16(sin_t) || !aligned16(y))
+    return SVDQ_ERR_ALIGN;
+  svdq_status st = device_info(nullptr, nullptr);
+  if (st != SVDQ_OK) return st;
+  NormRopeArgs a{y, norm_q, norm_k, cos_t, sin_t, M, heads, eps};
+  return from_cuda(launch_norm_rope(a, static_cast<cudaStream_t>(stream)));
+}
+
 svdq_status awq_pack_weight(int K, int N, const float* W, uint8_t* q, uint16_t* scales, uint16_t* zeros,
                             void* stream) {
   if (K <= 0 || N <= 0) return SVDQ_ERR_INVALID_ARG;
@@ -361,7 +409,7 @@ svdq_status svdq_probe_wait_timeout(unsigned long long limit_ns, void* stream) {
 }
 
 svdq_status svdq_probe_mma_peak(int iters, int mode, void* stream) {
-  if (iters < 1 || iters > (1 << 20) || (mode != 0 && mode != 1)) return SVDQ_ERR_INVALID_ARG;
+  if (iters < 1 || iters > (1 << 20) || mode < 0 || mode > 4) return SVDQ_ERR_INVALID_ARG;
   unsigned* err = nullptr;
   int sms = 0;
   svdq_status st = device_info(&err, &sms);

@@ -25,7 +25,10 @@
 //   warps 2..9  epilogue (both CTAs), two warps per TMEM lane quadrant, each
 //               draining half of the 256 columns: tcgen05.ld, y = alpha*acc +
 //               bias (read through the L1 cache), convert, stage 32 x 64
-//               pieces in 128B-swizzled shared memory, TMA store.
+//               pieces in 128B-swizzled shared memory, TMA store. With the
+//               fused QKV epilogue (svdq_w4a4_linear_qkv) a half is one head
+//               of 128 columns: Q and K heads are RMS-normalised and rotated
+//               before the store.
 // Accumulators: two 256-column buffers overlapping in 64 columns
 // ([0,256) and [192,448); scales in [448,512)). Per tile, the epilogue half
 // that holds the overlapped 64 columns drains them first and then releases
@@ -77,8 +80,76 @@ struct Params {
   int out_f32;
   unsigned* err;
   unsigned long long wait_ns;
+  // fused QKV epilogue (qkv_heads > 0): N = 3 * qkv_heads * 128, Q, K, V in
+  // that order; RMSNorm weights [128] of Q and K heads, eps, rotary tables
+  // cos/sin fp32 [M, 64]
+  int qkv_heads;
+  const uint16_t* norm_q;
+  const uint16_t* norm_k;
+  float eps;
+  const float* cos_t;
+  const float* sin_t;
 };
 
+// Output of 32 columns of a Q or K head (head columns hc0 .. hc0 + 31, in
+// registers as fp32 layer outputs y): u = y * inv * w, then the rotary
+// embedding of each adjacent pair (2i, 2i+1) by the row's angle i, rounded to
+// bf16 into 16-byte units u0 .. u0 + 3 of the 128B-swizzled staging row.
+__device__ __forceinline__ void qkv_out32(uint8_t* buf, int lane, const float (&y)[32], int hc0, int u0, float inv,
+                                          const uint16_t* w, const float* cos_row, const float* sin_row) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int hc = hc0 + 8 * u;  // head column of the 8 values
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w + hc));
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(cos_row + hc / 2));
+    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sin_row + hc / 2));
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+    const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+    uint32_t w4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a0 = y[8 * u + 2 * k] * inv * bf16_bits_to_f32(ww[k] & 0xFFFFu);
+      const float a1 = y[8 * u + 2 * k + 1] * inv * bf16_bits_to_f32(ww[k] >> 16);
+      const float o0 = fmaf(a0, cs[k], -a1 * sn[k]);
+      const float o1 = fmaf(a0, sn[k], a1 * cs[k]);
+      w4[k] = f32_to_bf16_bits(o0) | (f32_to_bf16_bits(o1) << 16);
+    }
+    *reinterpret_cast<uint4*>(buf + lane * 128 + (((u0 + u) ^ (lane & 7)) * 16)) =
+        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    // one unit's table loads at a time (keeps them from being hoisted into
+    // registers that the caller's live values need)
+    asm volatile("" ::: "memory");
+  }
+}
+
+// bf16 of 32 layer outputs into 16-byte units u0 .. u0 + 3 of the staging row
+__device__ __forceinline__ void plain_out32(uint8_t* buf, int lane, const float (&y)[32], int u0) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w4[k] = f32_to_bf16_bits(y[8 * u + 2 * k]) | (f32_to_bf16_bits(y[8 * u + 2 * k + 1]) << 16);
+    *reinterpret_cast<uint4*>(buf + lane * 128 + (((u0 + u) ^ (lane & 7)) * 16)) =
+        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+}
+
+// y = alpha * acc + bias of 32 consecutive columns starting at column n
+__device__ __forceinline__ void layer_out32(float (&y)[32], const uint32_t (&acc)[32], float alpha,
+                                            const uint16_t* bias, int n) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    const uint32_t bw = bias ? __ldg(reinterpret_cast<const uint32_t*>(bias + n + c)) : 0u;
+    y[c] = fmaf(alpha, __uint_as_float(acc[c]), bf16_bits_to_f32(bw & 0xFFFFu));
+    y[c + 1] = fmaf(alpha, __uint_as_float(acc[c + 1]), bf16_bits_to_f32(bw >> 16));
+  }
+}
+
+
+// kQkv: the fused QKV epilogue (a separate instance, so that the plain
+// GEMM's register allocation does not carry it).
+template <bool kQkv>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -281,6 +352,124 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       if (!mbar_wait(&sm.acc_full[b], (i >> 1) & 1, p.wait_ns, p.err)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (b ? kAccCol1 : kAccCol0) + 128 * h + ((uint32_t)(32 * q) << 16);
+      if constexpr (kQkv) {
+        // Fused QKV epilogue: the warp's half of the tile is one head of 128
+        // columns, 2 tn + h. A Q or K head is normalised over its 128 columns
+        // (RMSNorm of the layer output before its rounding) and rotated; a V
+        // head takes the plain epilogue below.
+        const int head = 2 * tn + h;
+        const int sect = head / p.qkv_heads;
+        const int cf = (b == 0 && h == 1) ? 1 : 0, cs = 1 - cf;  // chunk order: the shared columns first
+        if (sect >= 2 || head * 128 >= p.N) {
+          // V head (or past N): the layer output, 32 columns at a time
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {
+            const int c = part == 0 ? cf : cs;
+            const int nc = tn * BN + 128 * h + 64 * c;
+            if (lane == 0) bulk_wait_read<kSlots - 1>();
+            __syncwarp();
+            uint8_t* buf = sm.out[e][0];
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t v[32];
+              float t[32];
+              tmem_ld32(tbase + 64 * c + 32 * hh, v);
+              tmem_ld_wait();
+              tmem_regs_ready(v);
+              if (holds_overlap && part == 0 && hh == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(free_bar);
+              }
+              layer_out32(t, v, alpha, nc < p.N ? p.bias : nullptr, nc + 32 * hh);
+              plain_out32(buf, lane, t, 4 * hh);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < p.M && nc < p.N) tma_store_2d(&tm_y, buf, nc, row0);
+              bulk_commit();
+            }
+          }
+          continue;
+        }
+        {
+          const uint16_t* wn = sect == 0 ? p.norm_q : p.norm_k;
+          const int nh = head * 128;
+          const int m = row0 + lane;
+          const int mc = m < p.M ? m : p.M - 1;  // a row past M is not stored: read any valid one
+          const float* cos_row = p.cos_t + (size_t)mc * 64;
+          const float* sin_row = p.sin_t + (size_t)mc * 64;
+          // the 64-column chunk that holds the shared columns (when this warp
+          // holds them) first: its layer outputs stay in registers; the other
+          // chunk is read once for the sum of squares and again for the output
+          float ya[32], yb[32];
+          float ss = 0.f;
+          {
+            uint32_t v[32];
+            tmem_ld32(tbase + 64 * cf, v);
+            tmem_ld_wait();
+            tmem_regs_ready(v);
+            layer_out32(ya, v, alpha, p.bias, nh + 64 * cf);
+            tmem_ld32(tbase + 64 * cf + 32, v);
+            tmem_ld_wait();
+            tmem_regs_ready(v);
+            if (holds_overlap) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(free_bar);
+            }
+            layer_out32(yb, v, alpha, p.bias, nh + 64 * cf + 32);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ss = fmaf(yb[c], yb[c], fmaf(ya[c], ya[c], ss));
+          }
+#pragma unroll 1
+          for (int qq = 0; qq < 4; ++qq) {
+            uint32_t v16[16];
+            tmem_ld16(tbase + 64 * cs + 16 * qq, v16);
+            tmem_ld_wait();
+            tmem_regs_ready(v16);
+#pragma unroll
+            for (int c = 0; c < 16; c += 2) {
+              const uint32_t bw =
+                  p.bias ? __ldg(reinterpret_cast<const uint32_t*>(p.bias + nh + 64 * cs + 16 * qq + c)) : 0u;
+              const float t0 = fmaf(alpha, __uint_as_float(v16[c]), bf16_bits_to_f32(bw & 0xFFFFu));
+              const float t1 = fmaf(alpha, __uint_as_float(v16[c + 1]), bf16_bits_to_f32(bw >> 16));
+              ss = fmaf(t1, t1, fmaf(t0, t0, ss));
+            }
+          }
+          const float inv = rsqrtf(fmaf(ss, 1.0f / 128.0f, p.eps));
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {
+            if (lane == 0) bulk_wait_read<kSlots - 1>();
+            __syncwarp();
+            uint8_t* buf = sm.out[e][0];
+            if (part == 0) {
+              qkv_out32(buf, lane, ya, 64 * cf, 0, inv, wn, cos_row, sin_row);
+              qkv_out32(buf, lane, yb, 64 * cf + 32, 4, inv, wn, cos_row, sin_row);
+            } else {
+#pragma unroll 1
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t v[32];
+                float t[32];
+                tmem_ld32(tbase + 64 * cs + 32 * hh, v);
+                tmem_ld_wait();
+                tmem_regs_ready(v);
+                layer_out32(t, v, alpha, p.bias, nh + 64 * cs + 32 * hh);
+                qkv_out32(buf, lane, t, 64 * cs + 32 * hh, 4 * hh, inv, wn, cos_row, sin_row);
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < p.M) tma_store_2d(&tm_y, buf, nh + 64 * (part == 0 ? cf : cs), row0);
+              bulk_commit();
+            }
+          }
+          continue;
+        }
+      }
+      if constexpr (!kQkv)
       for (int step = 0; step < nchunks; ++step) {
         // buffer 0's upper half drains from its top, everything else from the
         // bottom: the shared columns come first
@@ -402,9 +591,16 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   p.out_f32 = a.out == 1;
   p.err = a.err;
   p.wait_ns = a.wait_ns;
+  p.qkv_heads = a.qkv_heads;
+  p.norm_q = a.norm_q;
+  p.norm_k = a.norm_k;
+  p.eps = a.eps;
+  p.cos_t = a.cos_t;
+  p.sin_t = a.sin_t;
 
   const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(gemm_nvfp4_kernel), (int)smem);
+  auto kern = p.qkv_heads > 0 ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;
   const int pairs = a.num_sms / 2;
@@ -419,7 +615,7 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, tm_a, tm_b, tm_sfa, tm_sfb, tm_p, tm_l, tm_y, p);
+  e = cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, tm_sfa, tm_sfb, tm_p, tm_l, tm_y, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

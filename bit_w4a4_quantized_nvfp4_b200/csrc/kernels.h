@@ -76,9 +76,27 @@ struct GemmArgs {
   unsigned* err;
   unsigned long long wait_ns;
   int num_sms;
+  // NVFP4 only: fused QKV epilogue when qkv_heads > 0 (head_dim 128)
+  int qkv_heads = 0;
+  const uint16_t* norm_q = nullptr;
+  const uint16_t* norm_k = nullptr;
+  float eps = 0.f;
+  const float* cos_t = nullptr;
+  const float* sin_t = nullptr;
 };
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_int4(const GemmArgs& a, cudaStream_t s);
+
+struct NormRopeArgs {
+  uint16_t* y;                // bf16 [M, 3 * heads * 128], Q and K sections updated in place
+  const uint16_t* norm_q;     // bf16 [128]
+  const uint16_t* norm_k;     // bf16 [128]
+  const float* cos_t;         // [M, 64]
+  const float* sin_t;         // [M, 64]
+  int M, heads;
+  float eps;
+};
+cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s);
 
 cudaError_t launch_probe_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3,
                                  uint16_t* bf16, cudaStream_t s);

@@ -7,10 +7,14 @@
 // issue and execution rate alone. It is the measured denominator of the
 // GEMM's roofline.
 //
-// mode 0: per 256-wide K stage, 4 MMAs (the GEMM's main loop without its
-//         operand stream);
-// mode 1: as 0, plus the 12 tcgen05.cp scale copies the GEMM issues per stage
-//         (shows what the scale copies cost the tensor pipe).
+// mode 0: per 256-wide K stage, 4 MMAs of N = 256 (the GEMM's main loop
+//         without its operand stream);
+// mode 1: as 0, plus 12 tcgen05.cp scale copies per stage (shows what the
+//         scale copies cost the tensor pipe);
+// mode 2: the same work as 8 MMAs of N = 128 per stage (two N halves);
+// mode 3: the same work as 16 MMAs of N = 64 per stage;
+// mode 4: as mode 2, but the 4 MMAs of each N half issued back to back into
+//         the same accumulator (instead of alternating the halves).
 #include "device.cuh"
 #include "kernels.h"
 
@@ -22,6 +26,8 @@ constexpr int kPStage = kPA + kPB + kPSfa + kPSfb;
 constexpr uint32_t kPSfaCol = 448, kPSfbCol = 464;
 // M = 256 (the pair), N = 256, E2M1 x E2M1 with UE4M3 scales per 16 (the GEMM's descriptor)
 constexpr uint32_t kPIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+constexpr uint32_t kPIdesc128 = (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+constexpr uint32_t kPIdesc64 = (1u << 7) | (1u << 10) | ((uint32_t)(64 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
 probe_mma_kernel(int iters, int mode, unsigned* err, unsigned long long wait_ns) {
@@ -80,10 +86,33 @@ probe_mma_kernel(int iters, int mode, unsigned* err, unsigned long long wait_ns)
             tc_cp_32x128b_warpx4_pair(tmem + kPSfbCol + 8 * j + 4, dcp[3 * j + 2]);
           }
         }
+        if (mode <= 1) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_nvfp4_pair(tmem, da[j], db[j], kPIdesc, tmem + kPSfaCol + 4 * j, tmem + kPSfbCol + 8 * j,
-                         (it > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < 4; ++j)
+            mma_nvfp4_pair(tmem, da[j], db[j], kPIdesc, tmem + kPSfaCol + 4 * j, tmem + kPSfbCol + 8 * j,
+                           (it > 0 || j > 0) ? 1u : 0u);
+        } else if (mode == 2) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+              mma_nvfp4_pair(tmem + 128 * hh, da[j], db[j] + (uint64_t)((64 * 128) >> 4) * hh, kPIdesc128,
+                             tmem + kPSfaCol + 4 * j, tmem + kPSfbCol + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
+        } else if (mode == 4) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              mma_nvfp4_pair(tmem + 128 * hh, da[j], db[j] + (uint64_t)((64 * 128) >> 4) * hh, kPIdesc128,
+                             tmem + kPSfaCol + 4 * j, tmem + kPSfbCol + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh)
+              mma_nvfp4_pair(tmem + 64 * hh, da[j], db[j] + (uint64_t)((32 * 128) >> 4) * hh, kPIdesc64,
+                             tmem + kPSfaCol + 4 * j, tmem + kPSfbCol + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
+        }
       }
       // both CTAs learn when every MMA has completed
       tc_commit_pair(&done, 0x3);

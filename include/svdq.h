@@ -151,6 +151,37 @@ svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const
                              const uint16_t* lr_up, const uint16_t* bias, void* y,
                              svdq_out_dtype out, void* stream);
 
+/* svdq_w4a4_linear_qkv — the NVFP4 layer as a grouped Q/K/V projection with
+ * the per-head RMSNorm of Q and K and the rotary embedding fused into the
+ * GEMM's epilogue (Diffusers "Nunchaku Lite" page, section on fused kernels:
+ * the QKV projection, RMSNorm and RoPE in one operator, and the grouped
+ * to_qkv linear with Q, K and V concatenated along the output dimension).
+ *   y_l = alpha * acc + P L2 + bias                      (as svdq_w4a4_linear, unrounded)
+ *   for each row m and each head of Q (weight norm_q) and of K (norm_k), head
+ *   columns d = 0..127:
+ *     u[d] = y_l[d] / sqrt(mean_d(y_l[d]^2) + eps) * w[d]
+ *     y[2i] = u[2i] cos[m,i] - u[2i+1] sin[m,i]; y[2i+1] = u[2i] sin[m,i] + u[2i+1] cos[m,i]
+ *   V heads: y = y_l. Output rounded to bf16 once.
+ * In:  as svdq_w4a4_linear (NVFP4); heads = heads per section (head_dim 128,
+ *      N = 3 * heads * 128); norm_q, norm_k bf16 [128]; eps >= 0; cos_t,
+ *      sin_t fp32 [M, 64] (row m = the token's angles for pairs i = 0..63).
+ * Out: y bf16 [M, N].
+ * Pointers 16-byte aligned (bias 4-byte). */
+svdq_status svdq_w4a4_linear_qkv(int M, int K, int heads, int r, const uint8_t* x_codes, const void* x_scales,
+                                 const uint16_t* P, const uint8_t* w_codes, const void* w_scales,
+                                 const float* w_tensor_scale, const uint16_t* lr_up, const uint16_t* bias,
+                                 const uint16_t* norm_q, const uint16_t* norm_k, float eps, const float* cos_t,
+                                 const float* sin_t, uint16_t* y, void* stream);
+
+/* svdq_qkv_norm_rope — the same per-head RMSNorm and rotary embedding as
+ * svdq_w4a4_linear_qkv, as a separate pass over a grouped Q/K/V projection's
+ * bf16 output y [M, 3 * heads * 128] (Q and K sections updated in place, V
+ * untouched). It reads the rounded output, so it is the unfused form of the
+ * operator that svdq_w4a4_linear_qkv computes on the unrounded accumulator.
+ * Arguments as svdq_w4a4_linear_qkv; pointers 16-byte aligned. */
+svdq_status svdq_qkv_norm_rope(int M, int heads, const uint16_t* norm_q, const uint16_t* norm_k, float eps,
+                               const float* cos_t, const float* sin_t, uint16_t* y, void* stream);
+
 /* awq_pack_weight — round-to-nearest asymmetric INT4 pack of W [K, N] with one
  * bf16 (scale, zero point) per output column and 64-block of K (Diffusers
  * "Nunchaku Lite" page, table "Supported quantization types", awq_w4a16):
@@ -207,9 +238,11 @@ svdq_status svdq_probe_wait_timeout(unsigned long long limit_ns, void* stream);
  * every CTA pair of the device (one pair per two SMs) issues `iters` K stages
  * of 4 block-scaled NVFP4 MMAs (tcgen05.mma.cta_group::2.kind::mxf4nvf4,
  * 256 x 256 x 64 each, the GEMM's instruction) on operands that stay in
- * shared memory: no loads, no epilogue. mode 1 also issues the GEMM's 12
- * scale copies (tcgen05.cp) per stage. The caller times the launch; the work
- * is (SMs/2) * iters * 4 * 2*256*256*64 FLOP. 1 <= iters <= 2^20. */
+ * shared memory: no loads, no epilogue. mode 1 also issues 12 scale copies
+ * (tcgen05.cp) per stage; modes 2 and 3 issue the same work as N = 128 or
+ * N = 64 MMAs (mode 4: the N = 128 MMAs of each half back to back into one
+ * accumulator). The caller times the launch; the work is
+ * (SMs/2) * iters * 4 * 2*256*256*64 FLOP. 1 <= iters <= 2^20, 0 <= mode <= 4. */
 svdq_status svdq_probe_mma_peak(int iters, int mode, void* stream);
 
 /* Test hook: pretend the device has compute capability major.minor (0, 0

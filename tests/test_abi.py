@@ -49,6 +49,7 @@ def test_status_strings(lib):
 def test_scale_sizes(lib):
     assert lib.svdq_scale_bytes(0, 256, 1024) == 256 * 64
     assert lib.svdq_scale_bytes(0, 200, 1024) == 256 * 64   # rows padded to 128
+    assert lib.svdq_scale_bytes(0, 300, 1024) == 384 * 64
     assert lib.svdq_scale_bytes(1, 200, 1024) == 200 * 16 * 2
     assert lib.svdq_scale_bytes(1, 200, 192) == 200 * 8 * 2  # INT4 row pitch: 3 groups padded to 8
     assert lib.svdq_scale_bytes(1, 7, 3072) == 7 * 48 * 2
@@ -203,3 +204,40 @@ def test_binding_checks_pack_and_awq(lib):
     bad = svdq.AwqWeight(128, 16, torch.zeros((16, 64), dtype=torch.uint8), _bf16(16, 1), _bf16(16, 2))
     _raises("w.scales", svdq.awq_w4a16_linear, _bf16(1, 128), bad)
     _raises("W: expected", svdq.awq_pack_weight, torch.zeros(128, 16, dtype=torch.float64))
+
+
+def test_qkv_entry_validation(lib):
+    S = svdq.Status
+    f = lib.svdq_w4a4_linear_qkv
+    # (M, K, heads, r, x_codes, x_scales, P, w_codes, w_scales, ts, lr_up, bias, nq, nk, eps, cos, sin, y, stream)
+    ok = [4, 64, 1, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1e-6, FAKE, FAKE, FAKE, None]
+
+    def call(**kw):
+        args = list(ok)
+        names = ["M", "K", "heads", "r", "xc", "xs", "P", "wc", "ws", "ts", "lr", "b", "nq", "nk", "eps", "cos",
+                 "sin", "y", "s"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+
+    assert call(heads=0) == S.INVALID_ARG
+    assert call(K=96) == S.SHAPE
+    assert call(eps=-1.0) == S.INVALID_ARG
+    assert call(nq=None) == S.INVALID_ARG
+    assert call(cos=None) == S.INVALID_ARG
+    assert call(r=16) == S.INVALID_ARG            # r > 0 needs P and lr_up
+    assert call(sin=FAKE + 4) == S.ALIGN
+    assert call(M=0, xc=None, xs=None, wc=None, ws=None, ts=None, nq=None, nk=None, cos=None, sin=None,
+                y=None) == S.OK
+
+
+def test_binding_checks_qkv(lib):
+    pw, qa = _packed(N=384), _act()
+    nq, nk = _bf16(128), _bf16(128)
+    cs, sn = torch.zeros(8, 64), torch.zeros(8, 64)
+    _raises("CUDA", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, cs, sn)   # well formed
+    _raises("3 \\* heads", svdq.w4a4_linear_qkv, qa, pw, 2, nq, nk, 1e-6, cs, sn)
+    _raises("norm_q: shape", svdq.w4a4_linear_qkv, qa, pw, 1, _bf16(64), nk, 1e-6, cs, sn)
+    _raises("cos: shape", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, torch.zeros(8, 32), sn)
+    _raises("NVFP4 only", svdq.w4a4_linear_qkv, _act(prec=svdq.INT4), _packed(prec=svdq.INT4, N=384), 1, nq, nk,
+            1e-6, cs, sn)

@@ -20,7 +20,7 @@ def _lib():
     svdq.load()
 
 
-@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 def test_mma_probe_runs(mode):
     svdq.probe_mma_peak(64, mode)
     torch.cuda.synchronize()
@@ -40,4 +40,4 @@ def test_mma_probe_rejects_bad_arguments():
     with pytest.raises(svdq.SvdqError):
         svdq.probe_mma_peak(0)
     with pytest.raises(svdq.SvdqError):
-        svdq.probe_mma_peak(16, mode=2)
+        svdq.probe_mma_peak(16, mode=5)

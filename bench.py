@@ -318,6 +318,9 @@ def run_cuda(args):
         out["cpu_baseline"] = cpu_baseline(d, rows=args.cpu_rows)
     if rank == 0 and not args.no_qkv:
         out["qkv_epilogue"] = bench_qkv(svdq, pw, L1, b, x, qa, flush, M, N, K)
+    if rank == 0 and not args.no_mlp:
+        del d
+        out["mlp_gelu"] = bench_mlp(svdq, flush)
     if rank == 0 and not args.no_awq:
         out["awq_gemv"] = [bench_awq(svdq, P, m) for m in synth.CONFIGS["c2_awq_gemv"]["Ms"]]
     if rank == 0 and not args.no_int4:
@@ -444,6 +447,70 @@ def bench_qkv(svdq, pw, L1, b, x, qa, flush, M, N, K, steps=30):
     res["speedup"] = round(res["unfused_ms"] / res["fused_ms"], 4)
     res["workload"] = (f"fused-QKV projection M{M} K{K} N{N} ({heads} heads of 128 per section) + RMSNorm of Q, K "
                        "+ rotary embedding")
+    return res
+
+
+def bench_mlp(svdq, flush, steps=30):
+    """The MLP pair of a DiT block at full size: up-projection 4608x3072 ->
+    12288, GELU, down-projection 4608x12288 -> 3072, both svdq_w4a4 NVFP4
+    layers with rank-32 branches. Fused: the up-projection's epilogue computes
+    GELU before its one rounding (bf16_gelu output) and its output is the
+    down-projection's activation-pass input (4 launches). Unfused: the plain
+    up-projection, then GELU as a separate elementwise pass (torch's
+    gelu, the non-fused stand-in), then the down-projection (4 launches + 1).
+    L2 flushed before each step; medians of CUDA-event times."""
+    up = synth.config_layer("c4_mlp_up_nvfp4")
+    down = synth.config_layer("c4_mlp_down_nvfp4")
+    M, K, F = up["M"], up["K"], up["N"]
+
+    def prep(d):
+        L1, L2 = bf16_dev(d["L1"]), bf16_dev(d["L2"])
+        pw = svdq.pack_weight("nvfp4", torch.from_numpy(d["W"]).cuda(), torch.from_numpy(d["lam"]).cuda(), L1, L2)
+        return pw, L1, bf16_dev(d["b"])
+
+    pw_u, L1u, bu = prep(up)
+    pw_d, L1d, bd = prep(down)
+    x = bf16_dev(up["x"])
+    qa_u = svdq.quantize_act(x, pw_u, L1u)
+    h = svdq.w4a4_linear(qa_u, pw_u, bu, out_dtype="bf16_gelu")
+    qa_d = svdq.quantize_act(h, pw_d, L1d)
+    y = svdq.w4a4_linear(qa_d, pw_d, bd)
+    yu = torch.empty_like(h)
+    torch.cuda.synchronize()
+
+    def fused():
+        svdq.quantize_act(x, pw_u, L1u, out=qa_u)
+        svdq.w4a4_linear(qa_u, pw_u, bu, out_dtype="bf16_gelu", out=h)
+        svdq.quantize_act(h, pw_d, L1d, out=qa_d)
+        svdq.w4a4_linear(qa_d, pw_d, bd, out=y)
+
+    def unfused():
+        svdq.quantize_act(x, pw_u, L1u, out=qa_u)
+        svdq.w4a4_linear(qa_u, pw_u, bu, out=yu)
+        hu = torch.nn.functional.gelu(yu, approximate="none")
+        svdq.quantize_act(hu, pw_d, L1d, out=qa_d)
+        svdq.w4a4_linear(qa_d, pw_d, bd, out=y)
+
+    res = {}
+    for name, fn in (("fused_ms", fused), ("unfused_ms", unfused)):
+        ts = []
+        for i in range(steps + 3):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1))
+        res[name] = round(statistics.median(ts), 5)
+    svdq.device_error()
+    flops = 2.0 * M * K * F * 2
+    res["fused_tflops"] = round(flops / (res["fused_ms"] * 1e-3) / 1e12, 1)
+    res["speedup"] = round(res["unfused_ms"] / res["fused_ms"], 4)
+    res["workload"] = (f"MLP pair M{M}: up K{K} -> N{F} (GELU) and down K{F} -> N{K}, NVFP4, r32 "
+                       "(seeded DiT-shaped inputs; the down-projection's input is the up-projection's output)")
+    res["unfused_gelu"] = "torch.nn.functional.gelu (erf) as a separate pass, the non-fused comparison"
     return res
 
 
@@ -642,6 +709,7 @@ def main():
     ap.add_argument("--no-int4", action="store_true")
     ap.add_argument("--no-probe", action="store_true")
     ap.add_argument("--no-qkv", action="store_true")
+    ap.add_argument("--no-mlp", action="store_true")
     ap.add_argument("--oracle-configs", action="store_true",
                     help="only time the CPU oracle on every workload (no GPU needed) and exit")
     args = ap.parse_args()

@@ -33,7 +33,7 @@ __all__ = [
 ]
 
 NVFP4, INT4 = 0, 1
-_OUT = {"bf16": 0, "f32": 1, "i32_groups": 2}
+_OUT = {"bf16": 0, "f32": 1, "i32_groups": 2, "bf16_gelu": 3}
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
 
@@ -280,11 +280,11 @@ def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = N
         _is(bias, torch.bfloat16, (N,), "bias")
     _need(out_dtype in _OUT, "out_dtype {!r}", out_dtype)
     want = {"bf16": (torch.bfloat16, (M, N)), "f32": (torch.float32, (M, N)),
-            "i32_groups": (torch.int32, (M, N, K // 64))}[out_dtype]
+            "i32_groups": (torch.int32, (M, N, K // 64)), "bf16_gelu": (torch.bfloat16, (M, N))}[out_dtype]
     if out is not None:
         _is(out, want[0], want[1], "out")
     if out is None:
-        if out_dtype == "bf16":
+        if out_dtype in ("bf16", "bf16_gelu"):
             out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.codes.device)
         elif out_dtype == "f32":
             out = torch.empty((M, N), dtype=torch.float32, device=qa.codes.device)

@@ -283,8 +283,10 @@ svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const
   if (st != SVDQ_OK) return st;
   if (M < 0 || N <= 0) return SVDQ_ERR_INVALID_ARG;
   if (N % 8) return SVDQ_ERR_SHAPE;
-  if (out != SVDQ_OUT_BF16 && out != SVDQ_OUT_F32 && out != SVDQ_OUT_I32_GROUPS) return SVDQ_ERR_INVALID_ARG;
+  if (out != SVDQ_OUT_BF16 && out != SVDQ_OUT_F32 && out != SVDQ_OUT_I32_GROUPS && out != SVDQ_OUT_BF16_GELU)
+    return SVDQ_ERR_INVALID_ARG;
   if (out == SVDQ_OUT_I32_GROUPS && p != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
+  if (out == SVDQ_OUT_BF16_GELU && p != SVDQ_NVFP4) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!x_codes || !x_scales || !w_codes || !w_scales || !w_tensor_scale || !y) return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!P || !lr_up)) return SVDQ_ERR_INVALID_ARG;

@@ -28,7 +28,9 @@
 //               pieces in 128B-swizzled shared memory, TMA store. With the
 //               fused QKV epilogue (svdq_w4a4_linear_qkv) a half is one head
 //               of 128 columns: Q and K heads are RMS-normalised and rotated
-//               before the store.
+//               before the store. With the GELU output mode the layer
+//               output goes through GELU before its rounding (the
+//               up-projection of the fused GELU-MLP).
 // Accumulators: two 256-column buffers overlapping in 64 columns
 // ([0,256) and [192,448); scales in [448,512)). Per tile, the epilogue half
 // that holds the overlapped 64 columns drains them first and then releases
@@ -147,9 +149,18 @@ __device__ __forceinline__ void layer_out32(float (&y)[32], const uint32_t (&acc
 }
 
 
-// kQkv: the fused QKV epilogue (a separate instance, so that the plain
-// GEMM's register allocation does not carry it).
-template <bool kQkv>
+// Epilogue of the instance: kEpiPlain (y = alpha acc + bias), kEpiQkv (the
+// fused QKV epilogue) or kEpiGelu (GELU of the layer output before its
+// rounding: the up-projection of the fused GELU-MLP). Separate instances, so
+// that the plain GEMM's register allocation carries neither.
+constexpr int kEpiPlain = 0, kEpiQkv = 1, kEpiGelu = 2;
+
+// GELU, erf form: y (1 + erf(y / sqrt 2)) / 2 in fp32
+__device__ __forceinline__ float gelu_erf(float y) {
+  return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
+}
+
+template <int kEpi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -352,7 +363,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       if (!mbar_wait(&sm.acc_full[b], (i >> 1) & 1, p.wait_ns, p.err)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + (b ? kAccCol1 : kAccCol0) + 128 * h + ((uint32_t)(32 * q) << 16);
-      if constexpr (kQkv) {
+      if constexpr (kEpi == kEpiQkv) {
         // Fused QKV epilogue: the warp's half of the tile is one head of 128
         // columns, 2 tn + h. A Q or K head is normalised over its 128 columns
         // (RMSNorm of the layer output before its rounding) and rotated; a V
@@ -469,7 +480,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           continue;
         }
       }
-      if constexpr (!kQkv)
+      if constexpr (kEpi != kEpiQkv)
       for (int step = 0; step < nchunks; ++step) {
         // buffer 0's upper half drains from its top, everything else from the
         // bottom: the shared columns come first
@@ -515,8 +526,12 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
               const int col = 8 * u + 2 * k;
               const uint32_t a0 = col < 32 ? v[col] : v2[col - 32];
               const uint32_t a1 = col + 1 < 32 ? v[col + 1] : v2[col + 1 - 32];
-              const float y0 = fmaf(alpha, __uint_as_float(a0), bb[2 * k]);
-              const float y1 = fmaf(alpha, __uint_as_float(a1), bb[2 * k + 1]);
+              float y0 = fmaf(alpha, __uint_as_float(a0), bb[2 * k]);
+              float y1 = fmaf(alpha, __uint_as_float(a1), bb[2 * k + 1]);
+              if constexpr (kEpi == kEpiGelu) {
+                y0 = gelu_erf(y0);
+                y1 = gelu_erf(y1);
+              }
               w4[k] = f32_to_bf16_bits(y0) | (f32_to_bf16_bits(y1) << 16);
             }
             *reinterpret_cast<uint4*>(buf + lane * 128 + ((u ^ (lane & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -599,7 +614,8 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   p.sin_t = a.sin_t;
 
   const size_t smem = sizeof(Smem) + 1024;
-  auto kern = p.qkv_heads > 0 ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
+  auto kern = p.qkv_heads > 0 ? gemm_nvfp4_kernel<kEpiQkv>
+                              : (a.out == 3 ? gemm_nvfp4_kernel<kEpiGelu> : gemm_nvfp4_kernel<kEpiPlain>);
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.tiles_m * p.tiles_n;

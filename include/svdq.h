@@ -63,7 +63,12 @@ typedef enum {
 typedef enum {
   SVDQ_OUT_BF16 = 0,      /* y as bf16 [M, N] (the layer output) */
   SVDQ_OUT_F32 = 1,       /* y as fp32 [M, N] before the final bf16 rounding */
-  SVDQ_OUT_I32_GROUPS = 2 /* INT4 only: raw int32 group dot products [M, N, K/64] */
+  SVDQ_OUT_I32_GROUPS = 2, /* INT4 only: raw int32 group dot products [M, N, K/64] */
+  SVDQ_OUT_BF16_GELU = 3   /* NVFP4 only: bf16 of GELU(y), erf form, of the unrounded
+                              output: the up-projection of the fused GELU-MLP
+                              (Diffusers "Nunchaku Lite" page, section on fused
+                              kernels), whose output feeds svdq_quantize_act of the
+                              down-projection directly */
 } svdq_out_dtype;
 
 /* Human-readable name of a status. Never NULL. */

@@ -83,6 +83,8 @@ def test_validation_rejects_before_any_device_access(lib):
     # linear
     assert lib.svdq_w4a4_linear(0, 4, 64, 8, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, 2, None) == S.INVALID_ARG
     assert lib.svdq_w4a4_linear(0, 4, 64, 8, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, 9, None) == S.INVALID_ARG
+    # the GELU output (fused GELU-MLP up-projection) is NVFP4 only
+    assert lib.svdq_w4a4_linear(1, 4, 64, 8, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, 3, None) == S.INVALID_ARG
     assert lib.svdq_w4a4_linear(0, 4, 64, 8, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, None, 0, None) == S.INVALID_ARG
     assert lib.svdq_w4a4_linear(0, 0, 64, 8, 0, None, None, None, None, None, None, None, None, None, 0, None) == S.OK
     assert lib.svdq_w4a4_linear(0, 4, 64, 8, 16, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, None, FAKE, 0, None) == S.INVALID_ARG

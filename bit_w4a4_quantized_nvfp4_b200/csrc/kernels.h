@@ -55,6 +55,8 @@ struct AwqArgs {
   int M, K, N;
 };
 cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
+// M = 1 or 2: the GEMV kernel (awq_gemv.cu); launch_awq dispatches to it
+cudaError_t launch_awq_gemv(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 
 // Row pitch, in scales, of the INT4 activation scales [M, K/64]: padded to a
 // multiple of 8 so that every row starts on a 16-byte boundary (the GEMM

@@ -58,7 +58,10 @@ def test_awq_gemv_full_size(full_weight, M):
     check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
 
 
-@pytest.mark.parametrize("M,K,N", [(3, 128, 72), (17, 192, 136), (40, 64, 8), (1, 4096, 24)])
+@pytest.mark.parametrize("M,K,N", [(3, 128, 72), (17, 192, 136), (40, 64, 8), (1, 4096, 24),
+                                   # one and two rows (the GEMV kernel): K not a whole number of
+                                   # 512-wide stages, an odd group count, N not a whole 64-row tile
+                                   (1, 320, 72), (2, 576, 200), (2, 64, 8), (1, 1088, 136), (2, 16384, 64)])
 def test_awq_ragged_shapes_with_bias(M, K, N):
     d = synth.awq_inputs(31, M, K, N)
     b = synth.bf16_bits(np.linspace(-0.05, 0.05, N))
@@ -137,3 +140,23 @@ def test_awq_reads_weights_written_just_before():
     y2 = svdq.awq_w4a16_linear(x, w)
     torch.cuda.synchronize()
     check_bf16_output(oracle.bf16_to_f32(bf16_np(y2)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_awq_gemv_outlier_activations(M):
+    """Activations with 1% of channels scaled x30 (as in the svdq workloads):
+    the one- and two-row kernel applies the zero point through activation
+    group sums, so large group sums must not cost accuracy."""
+    K, N = 3072, 512
+    d = synth.awq_inputs(52, M, K, N)
+    x = oracle.bf16_to_f32(d["x"]).astype(np.float64)
+    ch = np.random.default_rng(7).choice(K, K // 100, replace=False)
+    x[:, ch] *= 30.0
+    xb = synth.bf16_bits(x)
+    pk = oracle.awq_pack_weight(d["W"])
+    w = svdq.awq_pack_weight(torch.from_numpy(d["W"]).cuda())
+    y = svdq.awq_w4a16_linear(bf16_dev(xb), w)
+    torch.cuda.synchronize()
+    assert svdq.device_error() == 0
+    yo = oracle.awq_linear(xb, pk)
+    check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))

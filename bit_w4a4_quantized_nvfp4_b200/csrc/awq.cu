@@ -91,7 +91,7 @@ struct AwqLayout {
 __global__ void __launch_bounds__(kThreadsA, 2)
 awq_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* base = smem_align<1024>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = a.K, N = a.N, M = a.M;
   const int ng = K / 64;

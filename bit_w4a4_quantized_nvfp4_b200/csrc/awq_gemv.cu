@@ -4,37 +4,47 @@
 // memory-bound). The weight stream is the whole cost, so the arithmetic per
 // weight is cut to what the stream can hide:
 //
-// * Dequantisation without the zero point: each nibble q becomes the bf16 of
-//   128 + q with one mask-and-or (the 8 nibbles of a 32-bit word give four
-//   bf16 pairs (k, k+4) with three shifts and four and-or operations). The
-//   tensor cores then form C_g = sum_k (128 + q_k) x_k in fp32 over a group
-//   g of 64, and the group's exact result follows from the activation group
-//   sum X_g = sum_k x_k once per group:
-//       sum_k (q_k - z_g) x_k = C_g - (128 + z_g) X_g,
-//   y = sum_g s_g (C_g - (128 + z_g) X_g) + bias. Products (128 + q) x are
-//   exact in fp32; C_g is ~130 |X_g| in size, so fp32 accumulation costs
-//   about 2^-24 * 130 |X_g| per step, far below the bf16 output rounding.
+// * Unpacking in fp16 without any offset: a nibble at bits 0-3 (16-19) of a
+//   word, masked out, IS the fp16 subnormal q * 2^-24; one at bits 4-7
+//   (20-23) is 16 q * 2^-24. One shift by 8 brings the upper byte's nibbles
+//   down, so the 8 nibbles of a word give four fp16 pairs (k, k+4) with one
+//   shift and four and operations. The activations of the odd pairs are
+//   stored divided by 16, so every product is q x 2^-24, exact in fp32, and
+//   the tensor cores (mma.sync m16n8k16, f16 inputs, fp32 accumulation) form
+//   C_g = 2^-24 sum_k q_k x_k per group. The zero point needs the group sum
+//   X_g = sum_k x_k once per group:
+//       sum_k (q_k - z_g) x_k = 2^24 C_g - z_g X_g.
+// * Activations in fp16, exactly: every group of 64 values of a row is
+//   scaled by a power of two 2^e that puts its largest magnitude in
+//   [2^14, 2^15) (bf16 has 8 significant bits, fp16 11), and the group's
+//   result is scaled back by 2^-e together with the group scale.
 // * All eight columns of the MMA do useful work at M = 1: column c of the
-//   B operand (mma.sync m16n8k16, A = 16 weight rows) holds the activation
-//   entries of group c only (zeros elsewhere), so one accumulator tile
-//   collects eight groups' dot products at once and the per-group scale,
-//   zero point and X_g are applied once per 8 x 64 weights of a row, not per
-//   MMA. At M = 2 the columns are (row m, group) for four groups.
+//   B operand (A = 16 weight rows) holds the activations of group c only
+//   (zeros elsewhere), so one accumulator tile collects eight groups' dot
+//   products at once and each group's scale is applied once per 8 x 64
+//   weights of a row, not per MMA. At M = 2 the columns are (row m, group)
+//   for four groups. An MMA's result is ready some 90 cycles after issue,
+//   and the pipe takes one every ~8 cycles per SM sub-partition, so each
+//   warp keeps four independent accumulator chains and issues them
+//   interleaved (the MMAs are volatile, so their order is kept).
 //
-// Data movement as in the batched kernel: a producer warp streams 64-row x
-// 512-K weight stages (two 64 x 256-K boxes, 128-byte swizzle, 16 KB) through
-// a 4-stage TMA ring with full/empty mbarriers; two warp groups (stage
-// phases) take alternate stages, four row tiles of 16 rows each; the CTA's
-// activations, scales and zero points are bulk-copied into shared memory once.
-// With programmatic dependent launch every weight tile of the CTA is
-// prefetched into L2 before the wait for the previous kernel in the stream
-// (a prefetch only moves data closer, L2 being the point of coherence) and
-// nothing is read into the SM before it.
+// Data movement: a producer warp streams 64-row x 512-K weight stages (two
+// 64 x 256-K boxes, 128-byte swizzle, 16 KB) through a 4-stage TMA ring with
+// full/empty mbarriers; two warp groups (stage phases) take alternate stages,
+// four row tiles of 16 rows each; the CTA's activations, scales and zero
+// points are bulk-copied into shared memory once. With programmatic dependent
+// launch the CTA's first weight stages and its scales and zero points are
+// prefetched into L2 before the wait for the previous kernel in the stream (a
+// prefetch only moves data closer, L2 being the point of coherence) and
+// nothing is read into the SM before it; the later stages are prefetched
+// right after the first loads.
 //
 // K order inside a group: the lane that owns a group's 32 bytes of a row uses
 // its nibbles as pairs (8j+i, 8j+i+4), j = word, i = 0..3; every 8-element
-// block of x is stored as the bf16 pairs (0,4) (1,5) (2,6) (3,7) (the same
-// permutation the batched kernel uses), so the dot product is unchanged.
+// block of x is stored as the fp16 pairs (0,4) (1,5)/16 (2,6) (3,7)/16, so the
+// dot product is unchanged. The eight 16-byte blocks of group g sit at block
+// positions j ^ (g & 7), so that the lanes that read block j of eight groups
+// hit different banks; the lanes whose B entries are zero load nothing.
 #include "device.cuh"
 #include "kernels.h"
 
@@ -52,30 +62,46 @@ constexpr int kThreadsG = (kComputeWarpsG + 1) * 32;
 constexpr int kGemvSmemLimit = 232448;
 static_assert(kStagesG % kPhasesG == 0, "a stage is reused by one warp group only");
 
-__device__ __forceinline__ void mma_16816g(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                           uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// nibbles i and i+4 of w -> bf16x2 (128 + q_i, 128 + q_{i+4})
-template <int I>
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
-  return ((w >> (4 * I)) & 0x000F000Fu) | 0x43004300u;
-}
-
-__device__ __forceinline__ uint32_t word_of(const uint4& a, const uint4& b, int j) {
-  const uint4& v = j < 4 ? a : b;
-  const int i = j & 3;
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
-__device__ __forceinline__ uint32_t prmt_g(uint32_t a, uint32_t b, uint32_t sel) {
+// f16x2 of (hi, lo) rounded to nearest
+__device__ __forceinline__ uint32_t f16x2(float hi, float lo) {
   uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// the 8 nibbles of w (k = 0..7 of a run) -> fp16 pairs (q_i, q_{i+4}) x 2^-24
+// for i = 0, 2 and x 16 * 2^-24 for i = 1, 3 (subnormals, exact)
+struct Pairs {
+  uint32_t p[4];
+};
+__device__ __forceinline__ Pairs unpack8(uint32_t w) {
+  const uint32_t v = w >> 8;
+  Pairs r;
+  r.p[0] = w & 0x000F000Fu;
+  r.p[1] = w & 0x00F000F0u;
+  r.p[2] = v & 0x000F000Fu;
+  r.p[3] = v & 0x00F000F0u;
+  return r;
+}
+
+// 16 bytes of shared memory into v if pred, else v unchanged (its zeros stay)
+__device__ __forceinline__ void lds128_if(uint32_t (&v)[4], bool pred, uint32_t addr) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t@p ld.shared.v4.b32 {%0, %1, %2, %3}, [%5];\n\t}"
+      : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3])
+      : "r"((uint32_t)pred), "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
 struct GemvLayout {
@@ -83,18 +109,17 @@ struct GemvLayout {
   int ngp;       // groups of kp
   int x_pitch;   // bytes per activation row (2 kp)
   int sz_pitch;  // bytes per weight row of scales / zero points (2 ng)
-  int off_x, off_xs, off_s, off_z, off_zero, off_red, off_bar, total;
+  int off_x, off_xs, off_s, off_z, off_red, off_bar, total;
   __host__ __device__ GemvLayout(int M, int K) {
     kp = ((K + kStageKG - 1) / kStageKG) * kStageKG;
     ngp = kp / 64;
     x_pitch = 2 * kp;
     sz_pitch = 2 * (K / 64);
     off_x = kStagesG * kStageBytesG;
-    off_xs = off_x + M * x_pitch;                   // X_g sums, fp32 [M][ngp]
-    off_s = off_xs + ((M * ngp * 4 + 15) / 16) * 16;
+    off_xs = off_x + M * x_pitch;                   // {2^-e, X'} per (row, group), fp32 [M][ngp][2]
+    off_s = off_xs + M * ngp * 8;
     off_z = off_s + ((kRowsG * sz_pitch + 15) / 16) * 16;
-    off_zero = off_z + ((kRowsG * sz_pitch + 15) / 16) * 16;
-    off_red = off_zero + 128;
+    off_red = off_z + ((kRowsG * sz_pitch + 15) / 16) * 16;
     off_bar = off_red + (kPhasesG - 1) * 4 * 32 * 2 * 4;
     total = off_bar + 2 * kStagesG * 8 + 8 + 8;
   }
@@ -104,7 +129,7 @@ template <int M>
 __global__ void __launch_bounds__(kThreadsG, 2)
 awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* base = smem_align<1024>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = a.K, N = a.N;
   const int ng = K / 64;
@@ -112,15 +137,15 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   const int n0 = blockIdx.x * kRowsG;
   const GemvLayout L(M, K);
   uint8_t* xs = base + L.off_x;
-  float* xsum = reinterpret_cast<float*>(base + L.off_xs);
+  float2* xgs = reinterpret_cast<float2*>(base + L.off_xs);  // {2^-e, sum of the group's x 2^e}
   const uint16_t* ss = reinterpret_cast<const uint16_t*>(base + L.off_s);
   const uint16_t* zs = reinterpret_cast<const uint16_t*>(base + L.off_z);
-  uint8_t* zero = base + L.off_zero;
   float* red = reinterpret_cast<float*>(base + L.off_red);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + L.off_bar);
   uint64_t* empty = full + kStagesG;
   uint64_t* xbar = empty + kStagesG;
   int* abort_flag = reinterpret_cast<int*>(xbar + 1);
+  const uint32_t sz_bytes = (uint32_t)(min(kRowsG, N - n0) * L.sz_pitch);
 
   if (threadIdx.x == 0) launch_dependents();
   if (threadIdx.x == 0) {
@@ -134,12 +159,15 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   }
   if (warp == kComputeWarpsG && lane == 0) {
     // Only hints before the previous kernel in the stream has finished: the
-    // tensor map and every weight tile of this CTA are pulled towards L2.
+    // tensor map, the first weight stages and this CTA's scales and zero
+    // points are pulled towards L2.
     tma_prefetch_desc(&tm_q);
-    for (int c = 0; c < nst; ++c) {
+    for (int c = 0; c < nst && c < kStagesG; ++c) {
       tma_prefetch_l2_2d(&tm_q, c * (kStageKG / 2), n0);
       tma_prefetch_l2_2d(&tm_q, c * (kStageKG / 2) + 128, n0);
     }
+    bulk_prefetch_l2(a.s + (size_t)n0 * ng, sz_bytes);
+    bulk_prefetch_l2(a.z + (size_t)n0 * ng, sz_bytes);
   }
   __syncthreads();
   grid_dependency_wait();
@@ -156,12 +184,15 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
         tma_load_2d(dst, &tm_q, &full[s], cc * (kStageKG / 2), n0);
         tma_load_2d(dst + kBoxBytesG, &tm_q, &full[s], cc * (kStageKG / 2) + 128, n0);
       };
-      const uint32_t sz_bytes = (uint32_t)(min(kRowsG, N - n0) * L.sz_pitch);
       mbar_expect_tx(xbar, (uint32_t)(M * 2 * K) + 2 * sz_bytes);
+      for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
       bulk_load(base + L.off_s, a.s + (size_t)n0 * ng, sz_bytes, xbar);
       bulk_load(base + L.off_z, a.z + (size_t)n0 * ng, sz_bytes, xbar);
-      for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
       for (; c < nst && c < kStagesG; ++c) issue_stage(c);
+      for (int cc = kStagesG; cc < nst; ++cc) {
+        tma_prefetch_l2_2d(&tm_q, cc * (kStageKG / 2), n0);
+        tma_prefetch_l2_2d(&tm_q, cc * (kStageKG / 2) + 128, n0);
+      }
       for (; c < nst; ++c) {
         const int s = c % kStagesG;
         if (!mbar_wait(&empty[s], ((c / kStagesG) - 1) & 1, wait_ns, err)) {
@@ -182,31 +213,51 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   // ---------------------------------------------------------------- compute
   bool ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0, wait_ns, err));
   if (ok) {
-    // per (row, group): the group sum X_g in a fixed order, then the group's
-    // 64 values permuted in place into pair order; groups past K are zeros
-    for (int t = threadIdx.x; t < M * L.ngp; t += kComputeWarpsG * 32) {
-      const int m = t / L.ngp, g = t % L.ngp;
-      uint4* p = reinterpret_cast<uint4*>(xs + m * L.x_pitch + 128 * g);
-      float sum = 0.f;
-      if (g < ng) {
+    // per (row, group), eight threads of a warp, one 16-byte chunk (8
+    // values) each: 2^e from the group's largest magnitude, then the values
+    // as fp16 x 2^e (odd pairs / 16) in pair order, written back in place to
+    // chunk position j ^ (g & 7) (so that lanes reading chunk j of eight
+    // consecutive groups hit different banks), and the group's sum of x 2^e;
+    // groups past K are zeros
+    const int total = M * L.ngp * 8;
+    for (int base0 = 0; base0 < total; base0 += kComputeWarpsG * 32) {
+      const int idx = base0 + threadIdx.x;
+      const bool valid = idx < total;
+      const int j = idx & 7, gt = idx >> 3;
+      const int m = valid ? gt / L.ngp : 0, g = valid ? gt % L.ngp : 0;
+      const bool live = valid && g < ng;
+      uint4* grp = reinterpret_cast<uint4*>(xs + m * L.x_pitch + 128 * g);
+      const uint4 u = live ? grp[j] : make_uint4(0, 0, 0, 0);
+      // per-half unsigned maxima of the magnitude bits (bf16 order = magnitude order)
+      const uint32_t m2 = __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
+                                   __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu));
+      uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
+      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+      // bf16 biased exponent E: |x| < 2^(E - 126), so 2^(141 - E) puts the
+      // largest magnitude in [2^14, 2^15); clamped so both powers are normal
+      const int ex = min(max(141 - (int)(amax >> 7), -126), 126);
+      const float sc = __uint_as_float((uint32_t)(ex + 127) << 23);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      float v[8], gsum = 0.f;
 #pragma unroll
-        for (int b = 0; b < 8; b += 2) {
-          const uint4 u = p[b], v = p[b + 1];
-          const uint32_t w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) sum += bf16_bits_to_f32(w[e] & 0xFFFFu) + bf16_bits_to_f32(w[e] >> 16);
-          p[b] = make_uint4(prmt_g(u.x, u.z, 0x5410u), prmt_g(u.x, u.z, 0x7632u), prmt_g(u.y, u.w, 0x5410u),
-                            prmt_g(u.y, u.w, 0x7632u));
-          p[b + 1] = make_uint4(prmt_g(v.x, v.z, 0x5410u), prmt_g(v.x, v.z, 0x7632u), prmt_g(v.y, v.w, 0x5410u),
-                                prmt_g(v.y, v.w, 0x7632u));
-        }
-      } else {
-#pragma unroll
-        for (int b = 0; b < 8; ++b) p[b] = make_uint4(0, 0, 0, 0);
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu) * sc;
+        v[2 * e + 1] = bf16_bits_to_f32(w[e] >> 16) * sc;
       }
-      xsum[m * L.ngp + g] = sum;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) gsum += v[e];
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
+      gsum += __shfl_xor_sync(0xffffffffu, gsum, 4);
+      // every lane of the group has read its chunk (the shuffles above
+      // consumed the loaded values) before any lane overwrites one
+      if (valid)
+        grp[j ^ (g & 7)] = make_uint4(f16x2(v[4], v[0]), f16x2(v[5] * 0.0625f, v[1] * 0.0625f), f16x2(v[6], v[2]),
+                                      f16x2(v[7] * 0.0625f, v[3] * 0.0625f));
+      if (valid && j == 0) xgs[m * L.ngp + g] = make_float2(__uint_as_float((uint32_t)(127 - ex) << 23), gsum);
     }
-    if (threadIdx.x < 8) reinterpret_cast<uint4*>(zero)[threadIdx.x] = make_uint4(0, 0, 0, 0);
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarpsG * 32) : "memory");
 
@@ -214,26 +265,25 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   const int gid = lane >> 2, t = lane & 3;
   const int r_lo = rt * 16 + gid, r_hi = r_lo + 8;
   const int n_lo = n0 + r_lo, n_hi = n0 + r_hi;
-  // the two groups (columns 2t, 2t+1 of the accumulator tile) and the batch
-  // row this lane's accumulator values belong to
+  const int pl = r_lo * ng, ph = r_hi * ng;  // rows of the scale / zero-point tables
+  // the batch row this lane's accumulator columns 2t, 2t+1 belong to
   const int m_c = M == 1 ? 0 : (t >> 1);
   float tot_lo = 0.f, tot_hi = 0.f;
 
-  // apply one sub-block's scales, zero points and group sums: columns 2t, 2t+1
-  // of the tile are groups ga, ga + 1 (of batch row m_c)
+  // columns 2t, 2t+1 of the tile are groups ga, ga + 1 (of batch row m_c):
+  // y += s 2^-e (2^24 C - z X')
   auto finish = [&](const float (&c)[4], int ga) {
     const int gb = ga + 1;
     const int ga_c = min(ga, ng - 1), gb_c = min(gb, ng - 1);
-    const float xa = xsum[m_c * L.ngp + ga], xb = xsum[m_c * L.ngp + gb];
-    const int pl = r_lo * (L.sz_pitch / 2), ph = r_hi * (L.sz_pitch / 2);
-    const float s0 = bf16_bits_to_f32(ss[pl + ga_c]), s1 = bf16_bits_to_f32(ss[pl + gb_c]);
-    const float s2 = bf16_bits_to_f32(ss[ph + ga_c]), s3 = bf16_bits_to_f32(ss[ph + gb_c]);
-    const float z0 = bf16_bits_to_f32(zs[pl + ga_c]) + 128.f, z1 = bf16_bits_to_f32(zs[pl + gb_c]) + 128.f;
-    const float z2 = bf16_bits_to_f32(zs[ph + ga_c]) + 128.f, z3 = bf16_bits_to_f32(zs[ph + gb_c]) + 128.f;
-    tot_lo = fmaf(s0, fmaf(-z0, xa, c[0]), tot_lo);
-    tot_lo = fmaf(s1, fmaf(-z1, xb, c[1]), tot_lo);
-    tot_hi = fmaf(s2, fmaf(-z2, xa, c[2]), tot_hi);
-    tot_hi = fmaf(s3, fmaf(-z3, xb, c[3]), tot_hi);
+    const float2 xa = xgs[m_c * L.ngp + ga], xb = xgs[m_c * L.ngp + gb];
+    const float t0 = fmaf(16777216.f, c[0], -bf16_bits_to_f32(zs[pl + ga_c]) * xa.y);
+    const float t1 = fmaf(16777216.f, c[1], -bf16_bits_to_f32(zs[pl + gb_c]) * xb.y);
+    const float t2 = fmaf(16777216.f, c[2], -bf16_bits_to_f32(zs[ph + ga_c]) * xa.y);
+    const float t3 = fmaf(16777216.f, c[3], -bf16_bits_to_f32(zs[ph + gb_c]) * xb.y);
+    tot_lo = fmaf(bf16_bits_to_f32(ss[pl + ga_c]) * xa.x, t0, tot_lo);
+    tot_lo = fmaf(bf16_bits_to_f32(ss[pl + gb_c]) * xb.x, t1, tot_lo);
+    tot_hi = fmaf(bf16_bits_to_f32(ss[ph + ga_c]) * xa.x, t2, tot_hi);
+    tot_hi = fmaf(bf16_bits_to_f32(ss[ph + gb_c]) * xb.x, t3, tot_hi);
   };
   auto ld_w = [&](const uint8_t* box, int r, int ch) {
     return *reinterpret_cast<const uint4*>(box + r * 128 + ((ch ^ (r & 7)) << 4));
@@ -251,29 +301,40 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
     if constexpr (M == 1) {
       // lane (gid, t): rows r_lo, r_hi, groups t (box 0) and t + 4 (box 1);
       // B column gid holds group gid: lane (gid, t) supplies it in its first
-      // register when gid == t and in its second when gid == t + 4
-      const uint8_t* xa_src = gid == t ? xs + 128 * (g0 + t) : zero;
-      const uint8_t* xb_src = gid == t + 4 ? xs + 128 * (g0 + t + 4) : zero;
-      float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+      // register when gid == t and in its second when gid == t + 4, and zeros
+      // otherwise (those lanes load nothing)
+      const int ga = g0 + t, gb = g0 + t + 4;
+      const uint32_t xa_base = smem_u32(xs + 128 * ga), xb_base = smem_u32(xs + 128 * gb);
+      const bool a_act = gid == t, b_act = gid == t + 4;
+      // x blocks double-buffered: block j + 1 is loaded before block j's MMAs
+      uint32_t xa[2][4] = {}, xb[2][4] = {};
+      lds128_if(xa[0], a_act, xa_base + ((0 ^ (ga & 7)) << 4));
+      lds128_if(xb[0], b_act, xb_base + ((0 ^ (gb & 7)) << 4));
+      float acc[4][4] = {};
+      uint4 L0, H0, L1, H1;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // the 16-byte half h of each group's 32 bytes
-        const uint4 L0 = ld_w(st, r_lo, 2 * t + h), H0 = ld_w(st, r_hi, 2 * t + h);
-        const uint4 L1 = ld_w(st + kBoxBytesG, r_lo, 2 * t + h), H1 = ld_w(st + kBoxBytesG, r_hi, 2 * t + h);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int j = 4 * h + jj;
-          const uint4 xa = *reinterpret_cast<const uint4*>(xa_src + 16 * j);
-          const uint4 xb = *reinterpret_cast<const uint4*>(xb_src + 16 * j);
-          const uint32_t wl0 = word_of(L0, L0, jj), wh0 = word_of(H0, H0, jj);
-          const uint32_t wl1 = word_of(L1, L1, jj), wh1 = word_of(H1, H1, jj);
-          float(&acc)[4] = (j & 1) ? cb : ca;
-          mma_16816g(acc, nib_pair<0>(wl0), nib_pair<0>(wh0), nib_pair<0>(wl1), nib_pair<0>(wh1), xa.x, xb.x);
-          mma_16816g(acc, nib_pair<1>(wl0), nib_pair<1>(wh0), nib_pair<1>(wl1), nib_pair<1>(wh1), xa.y, xb.y);
-          mma_16816g(acc, nib_pair<2>(wl0), nib_pair<2>(wh0), nib_pair<2>(wl1), nib_pair<2>(wh1), xa.z, xb.z);
-          mma_16816g(acc, nib_pair<3>(wl0), nib_pair<3>(wh0), nib_pair<3>(wl1), nib_pair<3>(wh1), xa.w, xb.w);
+      for (int j = 0; j < 8; ++j) {
+        if ((j & 3) == 0) {  // the 16-byte half j / 4 of each group's 32 bytes
+          const int h = j >> 2;
+          L0 = ld_w(st, r_lo, 2 * t + h);
+          H0 = ld_w(st, r_hi, 2 * t + h);
+          L1 = ld_w(st + kBoxBytesG, r_lo, 2 * t + h);
+          H1 = ld_w(st + kBoxBytesG, r_hi, 2 * t + h);
         }
+        if (j + 1 < 8) {
+          lds128_if(xa[(j + 1) & 1], a_act, xa_base + (((j + 1) ^ (ga & 7)) << 4));
+          lds128_if(xb[(j + 1) & 1], b_act, xb_base + (((j + 1) ^ (gb & 7)) << 4));
+        }
+        const int jj = j & 3;
+        const Pairs al0 = unpack8(word_of(L0, jj)), ah0 = unpack8(word_of(H0, jj));
+        const Pairs al1 = unpack8(word_of(L1, jj)), ah1 = unpack8(word_of(H1, jj));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          mma_f16(acc[i], al0.p[i], ah0.p[i], al1.p[i], ah1.p[i], xa[j & 1][i], xb[j & 1][i]);
       }
-      const float cc[4] = {ca[0] + cb[0], ca[1] + cb[1], ca[2] + cb[2], ca[3] + cb[3]};
+      float cc[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cc[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
       keep = cc[0] + cc[1] + cc[2] + cc[3];
       finish(cc, g0 + 2 * t);
     } else {
@@ -283,18 +344,30 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
       for (int b = 0; b < 2; ++b) {
         const uint8_t* box = st + b * kBoxBytesG;
         const int gb0 = g0 + 4 * b;
-        const uint4 La = ld_w(box, r_lo, 2 * t), Lb = ld_w(box, r_lo, 2 * t + 1);
-        const uint4 Ha = ld_w(box, r_hi, 2 * t), Hb = ld_w(box, r_hi, 2 * t + 1);
-        const uint8_t* x_src = (gid & 3) == t ? xs + (gid >> 2) * L.x_pitch + 128 * (gb0 + t) : zero;
-        float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
+        const int gx = gb0 + t;
+        const uint32_t x_base = smem_u32(xs + (gid >> 2) * L.x_pitch + 128 * gx);
+        const bool act = (gid & 3) == t;
+        // x blocks double-buffered: block j + 1 is loaded before block j's MMAs
+        uint32_t v[2][4] = {};
+        lds128_if(v[0], act, x_base + ((0 ^ (gx & 7)) << 4));
+        float acc[4][4] = {};
+        uint4 Lw, Hw;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint4 v = *reinterpret_cast<const uint4*>(x_src + 16 * j);
-          const uint32_t wl = word_of(La, Lb, j), wh = word_of(Ha, Hb, j);
-          mma_16816g(ca, nib_pair<0>(wl), nib_pair<0>(wh), nib_pair<1>(wl), nib_pair<1>(wh), v.x, v.y);
-          mma_16816g(cb, nib_pair<2>(wl), nib_pair<2>(wh), nib_pair<3>(wl), nib_pair<3>(wh), v.z, v.w);
+          if ((j & 3) == 0) {
+            Lw = ld_w(box, r_lo, 2 * t + (j >> 2));
+            Hw = ld_w(box, r_hi, 2 * t + (j >> 2));
+          }
+          if (j + 1 < 8) lds128_if(v[(j + 1) & 1], act, x_base + (((j + 1) ^ (gx & 7)) << 4));
+          const int jj = j & 3;
+          const Pairs pl_ = unpack8(word_of(Lw, jj)), ph_ = unpack8(word_of(Hw, jj));
+          const uint32_t(&vv)[4] = v[j & 1];
+          mma_f16(acc[2 * (j & 1)], pl_.p[0], ph_.p[0], pl_.p[1], ph_.p[1], vv[0], vv[1]);
+          mma_f16(acc[2 * (j & 1) + 1], pl_.p[2], ph_.p[2], pl_.p[3], ph_.p[3], vv[2], vv[3]);
         }
-        const float cc[4] = {ca[0] + cb[0], ca[1] + cb[1], ca[2] + cb[2], ca[3] + cb[3]};
+        float cc[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cc[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
         keep += cc[0] + cc[1] + cc[2] + cc[3];
         finish(cc, gb0 + 2 * (t & 1));
       }
@@ -321,20 +394,20 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarpsG * 32) : "memory");
   if (*abort_flag || kh > 0) return;
 #pragma unroll
-  for (int ph = 1; ph < kPhasesG; ++ph) {
-    const float* rb = red + (size_t)((ph - 1) * 4 + rt) * 32 * 2;
+  for (int q = 1; q < kPhasesG; ++q) {
+    const float* rb = red + (size_t)((q - 1) * 4 + rt) * 32 * 2;
     tot_lo += rb[2 * lane];
     tot_hi += rb[2 * lane + 1];
   }
   const bool writer = M == 1 ? t == 0 : (t & 1) == 0;
   if (!writer) return;
   if (n_lo < N) {
-    const float b = a.bias ? bf16_bits_to_f32(a.bias[n_lo]) : 0.f;
-    a.y[(size_t)m_c * N + n_lo] = (uint16_t)f32_to_bf16_bits(__fadd_rn(tot_lo, b));
+    const float bb = a.bias ? bf16_bits_to_f32(a.bias[n_lo]) : 0.f;
+    a.y[(size_t)m_c * N + n_lo] = (uint16_t)f32_to_bf16_bits(__fadd_rn(tot_lo, bb));
   }
   if (n_hi < N) {
-    const float b = a.bias ? bf16_bits_to_f32(a.bias[n_hi]) : 0.f;
-    a.y[(size_t)m_c * N + n_hi] = (uint16_t)f32_to_bf16_bits(__fadd_rn(tot_hi, b));
+    const float bb = a.bias ? bf16_bits_to_f32(a.bias[n_hi]) : 0.f;
+    a.y[(size_t)m_c * N + n_hi] = (uint16_t)f32_to_bf16_bits(__fadd_rn(tot_hi, bb));
   }
 }
 

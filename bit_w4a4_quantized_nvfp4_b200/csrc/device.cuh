@@ -83,6 +83,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// The dynamic shared memory window rounded up to kAlign bytes. Computed by
+// pointer arithmetic on the extern array (no integer round trip), so that the
+// compiler still knows the result and everything derived from it to be shared
+// memory and compiles plain C++ accesses through it to shared-memory
+// instructions rather than generic ones.
+template <uint32_t kAlign>
+__device__ __forceinline__ uint8_t* smem_align(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return raw + ((kAlign - (a & (kAlign - 1))) & (kAlign - 1));
+}
+
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
   asm volatile(
@@ -220,6 +231,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Prefetch a contiguous range into L2 (a hint: no shared memory, no barrier);
+// address 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // --------------------------------------------------------------------------

@@ -123,7 +123,7 @@ gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constan
                  const __grid_constant__ CUtensorMap tm_xs, const __grid_constant__ CUtensorMap tm_ws,
                  const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  Smem& sm = *reinterpret_cast<Smem*>(smem_align<1024>(smem_raw));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int nblk = (p.NG + kScG - 1) / kScG;  // scale blocks per tile

@@ -32,7 +32,7 @@ constexpr uint32_t kPIdesc64 = (1u << 7) | (1u << 10) | ((uint32_t)(64 >> 3) << 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
 probe_mma_kernel(int iters, int mode, unsigned* err, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* st = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* st = smem_align<1024>(smem_raw);
   __shared__ uint64_t done;
   __shared__ uint32_t tmem_base;
   const int warp = threadIdx.x >> 5;

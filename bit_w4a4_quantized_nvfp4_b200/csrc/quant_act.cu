@@ -193,7 +193,7 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   constexpr int S = C::kStages;
   constexpr int CW = C::kConsumerWarps;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* base = smem_align<1024>(smem_raw);
   uint8_t* stages = base;                                       // S x kStageBytes
   uint64_t* full = reinterpret_cast<uint64_t*>(base + S * C::kStageBytes);
   uint64_t* empty = full + S;

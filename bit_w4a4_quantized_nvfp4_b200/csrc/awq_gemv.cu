@@ -213,50 +213,60 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   // ---------------------------------------------------------------- compute
   bool ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0, wait_ns, err));
   if (ok) {
-    // per (row, group), eight threads of a warp, one 16-byte chunk (8
+    // per (row, group), four threads of a warp, two 16-byte blocks (16
     // values) each: 2^e from the group's largest magnitude, then the values
     // as fp16 x 2^e (odd pairs / 16) in pair order, written back in place to
-    // chunk position j ^ (g & 7) (so that lanes reading chunk j of eight
+    // block position j ^ (g & 7) (so that lanes reading block j of eight
     // consecutive groups hit different banks), and the group's sum of x 2^e;
     // groups past K are zeros
-    const int total = M * L.ngp * 8;
+    const int total = M * L.ngp * 4;
     for (int base0 = 0; base0 < total; base0 += kComputeWarpsG * 32) {
       const int idx = base0 + threadIdx.x;
       const bool valid = idx < total;
-      const int j = idx & 7, gt = idx >> 3;
+      const int jp = idx & 3, gt = idx >> 2;
       const int m = valid ? gt / L.ngp : 0, g = valid ? gt % L.ngp : 0;
       const bool live = valid && g < ng;
       uint4* grp = reinterpret_cast<uint4*>(xs + m * L.x_pitch + 128 * g);
-      const uint4 u = live ? grp[j] : make_uint4(0, 0, 0, 0);
+      uint4 u[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) u[h] = live ? grp[2 * jp + h] : make_uint4(0, 0, 0, 0);
       // per-half unsigned maxima of the magnitude bits (bf16 order = magnitude order)
-      const uint32_t m2 = __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
-                                   __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu));
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(u[h].x & 0x7FFF7FFFu, u[h].y & 0x7FFF7FFFu),
+                                   __vmaxu2(u[h].z & 0x7FFF7FFFu, u[h].w & 0x7FFF7FFFu)));
       uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
       amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
       // bf16 biased exponent E: |x| < 2^(E - 126), so 2^(141 - E) puts the
       // largest magnitude in [2^14, 2^15); clamped so both powers are normal
       const int ex = min(max(141 - (int)(amax >> 7), -126), 126);
       const float sc = __uint_as_float((uint32_t)(ex + 127) << 23);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-      float v[8], gsum = 0.f;
+      uint4 outv[2];
+      float gsum = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        v[2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu) * sc;
-        v[2 * e + 1] = bf16_bits_to_f32(w[e] >> 16) * sc;
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t w[4] = {u[h].x, u[h].y, u[h].z, u[h].w};
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] = bf16_bits_to_f32(w[e] & 0xFFFFu) * sc;
+          v[2 * e + 1] = bf16_bits_to_f32(w[e] >> 16) * sc;
+        }
+        gsum += ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+        outv[h] = make_uint4(f16x2(v[4], v[0]), f16x2(v[5] * 0.0625f, v[1] * 0.0625f), f16x2(v[6], v[2]),
+                             f16x2(v[7] * 0.0625f, v[3] * 0.0625f));
       }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) gsum += v[e];
       gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
       gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
-      gsum += __shfl_xor_sync(0xffffffffu, gsum, 4);
-      // every lane of the group has read its chunk (the shuffles above
+      // every lane of the group has read its blocks (the shuffles above
       // consumed the loaded values) before any lane overwrites one
-      if (valid)
-        grp[j ^ (g & 7)] = make_uint4(f16x2(v[4], v[0]), f16x2(v[5] * 0.0625f, v[1] * 0.0625f), f16x2(v[6], v[2]),
-                                      f16x2(v[7] * 0.0625f, v[3] * 0.0625f));
-      if (valid && j == 0) xgs[m * L.ngp + g] = make_float2(__uint_as_float((uint32_t)(127 - ex) << 23), gsum);
+      if (valid) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) grp[(2 * jp + h) ^ (g & 7)] = outv[h];
+      }
+      if (valid && jp == 0) xgs[m * L.ngp + g] = make_float2(__uint_as_float((uint32_t)(127 - ex) << 23), gsum);
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarpsG * 32) : "memory");

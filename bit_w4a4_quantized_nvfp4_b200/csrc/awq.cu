@@ -339,9 +339,9 @@ int awq_rows_per_launch(int K) {
 }
 
 cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s) {
-  // one or two rows: the GEMV kernel, whose MMA columns hold groups rather
-  // than batch rows
-  if (a.M <= 2) return launch_awq_gemv(a, err, wait_ns, s);
+  // up to four rows: the GEMV kernel, whose MMA columns hold groups as well as
+  // batch rows (when its shared memory plan fits the row length)
+  if (awq_gemv_fits(a.M, a.K)) return launch_awq_gemv(a, err, wait_ns, s);
   CUtensorMap tm_q;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q, (uint64_t)a.K / 2, (uint64_t)a.N, (uint64_t)a.K / 2,
                     kStageK / 2, kRowsA, CU_TENSOR_MAP_SWIZZLE_128B))

@@ -125,7 +125,10 @@ struct GemvLayout {
   }
 };
 
-template <int M>
+// MT = 1, 2 or 4: the rows of the MMA's eight columns (eight groups per
+// column block at MT = 1, four at MT = 2, two at MT = 4); the launch's a.M <= MT
+// rows are real, the rest zeros.
+template <int MT>
 __global__ void __launch_bounds__(kThreadsG, 2)
 awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* err, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
@@ -135,7 +138,8 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   const int ng = K / 64;
   const int nst = (K + kStageKG - 1) / kStageKG;
   const int n0 = blockIdx.x * kRowsG;
-  const GemvLayout L(M, K);
+  const int M = a.M;
+  const GemvLayout L(MT, K);
   uint8_t* xs = base + L.off_x;
   float2* xgs = reinterpret_cast<float2*>(base + L.off_xs);  // {2^-e, sum of the group's x 2^e}
   const uint16_t* ss = reinterpret_cast<const uint16_t*>(base + L.off_s);
@@ -219,13 +223,13 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
     // block position j ^ (g & 7) (so that lanes reading block j of eight
     // consecutive groups hit different banks), and the group's sum of x 2^e;
     // groups past K are zeros
-    const int total = M * L.ngp * 4;
+    const int total = MT * L.ngp * 4;
     for (int base0 = 0; base0 < total; base0 += kComputeWarpsG * 32) {
       const int idx = base0 + threadIdx.x;
       const bool valid = idx < total;
       const int jp = idx & 3, gt = idx >> 2;
       const int m = valid ? gt / L.ngp : 0, g = valid ? gt % L.ngp : 0;
-      const bool live = valid && g < ng;
+      const bool live = valid && g < ng && m < M;
       uint4* grp = reinterpret_cast<uint4*>(xs + m * L.x_pitch + 128 * g);
       uint4 u[2];
 #pragma unroll
@@ -276,14 +280,18 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   const int r_lo = rt * 16 + gid, r_hi = r_lo + 8;
   const int n_lo = n0 + r_lo, n_hi = n0 + r_hi;
   const int pl = r_lo * ng, ph = r_hi * ng;  // rows of the scale / zero-point tables
-  // the batch row this lane's accumulator columns 2t, 2t+1 belong to
-  const int m_c = M == 1 ? 0 : (t >> 1);
+  // Column c of the accumulator tile is batch row c / G, group c % G of the
+  // column block. This lane's columns 2t and 2t + 1: at G >= 2 both in batch
+  // row m_c (groups 2t % G and 2t % G + 1).
+  constexpr int G = 8 / MT;
+  const int m_c = (2 * t) / G;
+  const int gi0 = (2 * t) % G;
   float tot_lo = 0.f, tot_hi = 0.f;
 
-  // columns 2t, 2t+1 of the tile are groups ga, ga + 1 (of batch row m_c):
-  // y += s 2^-e (2^24 C - z X')
-  auto finish = [&](const float (&c)[4], int ga) {
-    const int gb = ga + 1;
+  // columns 2t, 2t+1 of the tile are groups ga, ga + 1 of the block starting
+  // at group gb0 (batch row m_c): y += s 2^-e (2^24 C - z X')
+  auto finish = [&](const float (&c)[4], int gb0) {
+    const int ga = gb0 + gi0, gb = ga + 1;
     const int ga_c = min(ga, ng - 1), gb_c = min(gb, ng - 1);
     const float2 xa = xgs[m_c * L.ngp + ga], xb = xgs[m_c * L.ngp + gb];
     const float t0 = fmaf(16777216.f, c[0], -bf16_bits_to_f32(zs[pl + ga_c]) * xa.y);
@@ -308,7 +316,7 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
     const uint8_t* st = base + s * kStageBytesG;
     const int g0 = c * 8;
     float keep = 0.f;
-    if constexpr (M == 1) {
+    if constexpr (MT == 1) {
       // lane (gid, t): rows r_lo, r_hi, groups t (box 0) and t + 4 (box 1);
       // B column gid holds group gid: lane (gid, t) supplies it in its first
       // register when gid == t and in its second when gid == t + 4, and zeros
@@ -346,29 +354,38 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
 #pragma unroll
       for (int e = 0; e < 4; ++e) cc[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
       keep = cc[0] + cc[1] + cc[2] + cc[3];
-      finish(cc, g0 + 2 * t);
+      finish(cc, g0);
     } else {
-      // two sub-blocks of four groups (one box each); lane (gid, t): rows
-      // r_lo, r_hi, group t of the box; B column gid = (row gid / 4, group gid % 4)
+      // blocks of G groups (8 / G per stage, each inside one box). Lane
+      // (gid, t): rows r_lo, r_hi, group gl = t % G of the block, share
+      // sigma = t / G of that group's 8 words (W = 2G words: all of them at
+      // G = 4, half at G = 2). B column gid = (batch row gid / G, group
+      // gid % G): lane (gid, t) supplies the activations of its slot pairs
+      // when gid % G == gl, from the same share.
+      constexpr int W = 2 * G;
+      const int gl = t % G, sigma = t / G;
+      const bool act = (gid % G) == gl;
+      const int xm = gid / G;
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const uint8_t* box = st + b * kBoxBytesG;
-        const int gb0 = g0 + 4 * b;
-        const int gx = gb0 + t;
-        const uint32_t x_base = smem_u32(xs + (gid >> 2) * L.x_pitch + 128 * gx);
-        const bool act = (gid & 3) == t;
+      for (int kbl = 0; kbl < 8 / G; ++kbl) {
+        const int gb0 = g0 + G * kbl;
+        const uint8_t* box = st + ((G * kbl) >> 2) * kBoxBytesG;
+        const int gib = ((G * kbl) & 3) + gl;  // the lane's group within the box
+        const int gx = gb0 + gl;
+        const uint32_t x_base = smem_u32(xs + xm * L.x_pitch + 128 * gx);
         // x blocks double-buffered: block j + 1 is loaded before block j's MMAs
         uint32_t v[2][4] = {};
-        lds128_if(v[0], act, x_base + ((0 ^ (gx & 7)) << 4));
+        lds128_if(v[0], act, x_base + (((sigma * W) ^ (gx & 7)) << 4));
         float acc[4][4] = {};
         uint4 Lw, Hw;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if ((j & 3) == 0) {
-            Lw = ld_w(box, r_lo, 2 * t + (j >> 2));
-            Hw = ld_w(box, r_hi, 2 * t + (j >> 2));
+        for (int j = 0; j < W; ++j) {
+          if ((j & 3) == 0) {  // the 16-byte chunk holding words sigma W + j ..
+            const int ch = 2 * gib + (sigma * W + j) / 4;
+            Lw = ld_w(box, r_lo, ch);
+            Hw = ld_w(box, r_hi, ch);
           }
-          if (j + 1 < 8) lds128_if(v[(j + 1) & 1], act, x_base + (((j + 1) ^ (gx & 7)) << 4));
+          if (j + 1 < W) lds128_if(v[(j + 1) & 1], act, x_base + (((sigma * W + j + 1) ^ (gx & 7)) << 4));
           const int jj = j & 3;
           const Pairs pl_ = unpack8(word_of(Lw, jj)), ph_ = unpack8(word_of(Hw, jj));
           const uint32_t(&vv)[4] = v[j & 1];
@@ -379,7 +396,7 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
 #pragma unroll
         for (int e = 0; e < 4; ++e) cc[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
         keep += cc[0] + cc[1] + cc[2] + cc[3];
-        finish(cc, gb0 + 2 * (t & 1));
+        finish(cc, gb0);
       }
     }
     // release the stage only once its weights have gone through the MMAs
@@ -388,10 +405,13 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  // lanes of one row and batch row: M = 1 all four of a quad, M = 2 pairs
-  tot_lo += __shfl_xor_sync(0xffffffffu, tot_lo, 1);
-  tot_hi += __shfl_xor_sync(0xffffffffu, tot_hi, 1);
-  if constexpr (M == 1) {
+  // lanes of one row and batch row: MT = 1 all four of a quad, MT = 2 pairs,
+  // MT = 4 each lane its own batch row
+  if constexpr (MT <= 2) {
+    tot_lo += __shfl_xor_sync(0xffffffffu, tot_lo, 1);
+    tot_hi += __shfl_xor_sync(0xffffffffu, tot_hi, 1);
+  }
+  if constexpr (MT == 1) {
     tot_lo += __shfl_xor_sync(0xffffffffu, tot_lo, 2);
     tot_hi += __shfl_xor_sync(0xffffffffu, tot_hi, 2);
   }
@@ -409,7 +429,7 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
     tot_lo += rb[2 * lane];
     tot_hi += rb[2 * lane + 1];
   }
-  const bool writer = M == 1 ? t == 0 : (t & 1) == 0;
+  const bool writer = (2 * t) % G == 0 && m_c < M;
   if (!writer) return;
   if (n_lo < N) {
     const float bb = a.bias ? bf16_bits_to_f32(a.bias[n_lo]) : 0.f;
@@ -423,15 +443,21 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
 
 }  // namespace
 
+static int gemv_rows(int M) { return M <= 2 ? M : 4; }
+
+bool awq_gemv_fits(int M, int K) {
+  return M >= 1 && M <= 4 && (size_t)GemvLayout(gemv_rows(M), K).total + 1024 <= (size_t)kGemvSmemLimit;
+}
+
 cudaError_t launch_awq_gemv(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s) {
-  if (a.M < 1 || a.M > 2) return cudaErrorInvalidValue;
+  if (!awq_gemv_fits(a.M, a.K)) return cudaErrorInvalidValue;
+  const int mt = gemv_rows(a.M);
   CUtensorMap tm_q;
   if (!make_tmap_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q, (uint64_t)a.K / 2, (uint64_t)a.N, (uint64_t)a.K / 2,
                     128, kRowsG, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const size_t smem = (size_t)GemvLayout(a.M, a.K).total + 1024;
-  if (smem > (size_t)kGemvSmemLimit) return cudaErrorInvalidValue;
-  auto kern = a.M == 1 ? awq_gemv_kernel<1> : awq_gemv_kernel<2>;
+  const size_t smem = (size_t)GemvLayout(mt, a.K).total + 1024;
+  auto kern = mt == 1 ? awq_gemv_kernel<1> : (mt == 2 ? awq_gemv_kernel<2> : awq_gemv_kernel<4>);
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

@@ -55,7 +55,9 @@ struct AwqArgs {
   int M, K, N;
 };
 cudaError_t launch_awq(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
-// M = 1 or 2: the GEMV kernel (awq_gemv.cu); launch_awq dispatches to it
+// M = 1..4: the GEMV kernel (awq_gemv.cu), when awq_gemv_fits(M, K);
+// launch_awq dispatches to it
+bool awq_gemv_fits(int M, int K);
 cudaError_t launch_awq_gemv(const AwqArgs& a, unsigned* err, unsigned long long wait_ns, cudaStream_t s);
 
 // Row pitch, in scales, of the INT4 activation scales [M, K/64]: padded to a

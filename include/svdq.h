@@ -205,10 +205,11 @@ svdq_status awq_pack_weight(int K, int N, const float* W, uint8_t* q, uint16_t* 
  * Out: y bf16 [M, N].
  * Shapes: K % 64 == 0, K <= 16384 (the activations of a block of rows are
  * held in shared memory), N % 8 == 0, M >= 0.
- * M = 1 or 2 runs the GEMV kernel: each group's dot product is formed with
+ * M = 1..4 runs the GEMV kernel (M = 3, 4 only while its shared-memory plan
+ * fits K; otherwise the batched kernel): each group's dot product is formed with
  * exact products in fp32 (the activations scaled into fp16 by a power of two
  * per group and row, the weight nibbles as exact fp16 values) and the zero
- * point applied once per group through the activation group sum; M >= 3 runs
+ * point applied once per group through the activation group sum; larger M runs
  * the batched kernel, which subtracts the zero point before its MMAs. Both
  * meet the same output tolerance; they may differ from each other in the
  * last bits of the fp32 sums (summation order).

@@ -59,9 +59,12 @@ def test_awq_gemv_full_size(full_weight, M):
 
 
 @pytest.mark.parametrize("M,K,N", [(3, 128, 72), (17, 192, 136), (40, 64, 8), (1, 4096, 24),
-                                   # one and two rows (the GEMV kernel): K not a whole number of
-                                   # 512-wide stages, an odd group count, N not a whole 64-row tile
-                                   (1, 320, 72), (2, 576, 200), (2, 64, 8), (1, 1088, 136), (2, 16384, 64)])
+                                   # one to four rows (the GEMV kernel): K not a whole number of
+                                   # 512-wide stages, an odd group count, N not a whole 64-row tile;
+                                   # three rows (the fourth MMA row zero); four rows at K = 16384
+                                   # (shared memory too small for the GEMV: the batched kernel)
+                                   (1, 320, 72), (2, 576, 200), (2, 64, 8), (1, 1088, 136), (2, 16384, 64),
+                                   (3, 320, 72), (4, 576, 200), (4, 64, 8), (3, 1088, 136), (4, 16384, 64)])
 def test_awq_ragged_shapes_with_bias(M, K, N):
     d = synth.awq_inputs(31, M, K, N)
     b = synth.bf16_bits(np.linspace(-0.05, 0.05, N))
@@ -142,11 +145,11 @@ def test_awq_reads_weights_written_just_before():
     check_bf16_output(oracle.bf16_to_f32(bf16_np(y2)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
 
 
-@pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
 def test_awq_gemv_outlier_activations(M):
     """Activations with 1% of channels scaled x30 (as in the svdq workloads):
-    the one- and two-row kernel applies the zero point through activation
-    group sums, so large group sums must not cost accuracy."""
+    the GEMV kernel (up to four rows) applies the zero point through
+    activation group sums, so large group sums must not cost accuracy."""
     K, N = 3072, 512
     d = synth.awq_inputs(52, M, K, N)
     x = oracle.bf16_to_f32(d["x"]).astype(np.float64)

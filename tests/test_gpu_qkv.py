@@ -77,7 +77,7 @@ def test_qkv_epilogue_c3_full_size():
     c = synth.CONFIGS["c3_qkv_nvfp4"]
     d = synth.config_layer("c3_qkv_nvfp4")
     e = synth.qkv_epilogue_inputs(c["seed"], c["M"], 128, c["N"] // 384)
-    rows = np.sort(np.random.default_rng(11).choice(c["M"], 128, replace=False)).astype(np.int32)
+    rows = np.sort(np.random.default_rng(11).choice(c["M"], 512, replace=False)).astype(np.int32)
     run_case(d, e, c["N"] // 384, rows=rows)
 
 

@@ -171,11 +171,11 @@ def test_full_size_workload_sampled_rows(name):
     both projections of the MLP pair (4608x3072 -> 12288 and, on GELU inputs,
     4608x12288 -> 3072; the K = 12288 activation pass walks 48 chunks, four
     times the QKV's). Weight and activation codes and scales and P are compared
-    in full, y on 160 seeded rows (the oracle computes those one by one)."""
+    in full, y on 512 seeded rows (the oracle computes those one by one)."""
     c = dict(synth.CONFIGS[name])
     d = synth.config_layer(name)
     pw, qa, y = run_layer("nvfp4", d)
-    rows = np.sort(np.random.default_rng(3).choice(c["M"], 160, replace=False)).astype(np.int32)
+    rows = np.sort(np.random.default_rng(3).choice(c["M"], 512, replace=False)).astype(np.int32)
     w, a, yo = oracle_layer("nvfp4", d, rows=rows)
     compare_pack_and_act("nvfp4", d, pw, qa, w, a)
     check_bf16_output(as_f32(bf16_np(y))[rows], yo, as_f32(oracle.bf16_rn(yo)))
@@ -276,11 +276,11 @@ def test_int4_linear_matches_oracle(M, K, N, r):
 
 def test_c5_int4_full_size():
     """INT4 workload (M4608 K3072 N9216 r32, g64): codes and scales in full, y
-    on 128 seeded rows, exact int32 group sums on the first 48 rows."""
+    on 512 seeded rows, exact int32 group sums on the first 48 rows."""
     c = synth.CONFIGS["c5_qkv_int4"]
     d = synth.config_layer("c5_qkv_int4")
     pw, qa, y = run_layer("int4", d)
-    rows = np.sort(np.random.default_rng(5).choice(c["M"], 128, replace=False)).astype(np.int32)
+    rows = np.sort(np.random.default_rng(5).choice(c["M"], 512, replace=False)).astype(np.int32)
     w, a, yo = oracle_layer("int4", d, rows=rows)
     compare_pack_and_act("int4", d, pw, qa, w, a)
     check_bf16_output(as_f32(bf16_np(y))[rows], yo, as_f32(oracle.bf16_rn(yo)))

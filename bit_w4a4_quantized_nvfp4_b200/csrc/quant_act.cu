@@ -221,7 +221,9 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   if (warp == CW && lane == 0) {
     tma_prefetch_desc(&tm_x);
     if (NT) tma_prefetch_desc(&tm_l1);
-    for (int c = 0; c < nchunks && c < S; ++c)
+    // only the first two chunks: a deeper prefetch (all S stages) queues ahead
+    // of the first chunk's own loads and delays the start (measured)
+    for (int c = 0; c < nchunks && c < 2; ++c)
       for (int b = 0; b < min(kChunk, K - c * kChunk) / 64; ++b) tma_prefetch_l2_2d(&tm_x, c * kChunk + 64 * b, row0);
   }
   // every input may be the previous kernel's output, every output may still

@@ -97,16 +97,33 @@ struct Params {
 // registers as fp32 layer outputs y): u = y * inv * w, then the rotary
 // embedding of each adjacent pair (2i, 2i+1) by the row's angle i, rounded to
 // bf16 into 16-byte units u0 .. u0 + 3 of the 128B-swizzled staging row.
-__device__ __forceinline__ void qkv_out32(uint8_t* buf, int lane, const float (&y)[32], int hc0, int u0, float inv,
-                                          const uint16_t* w, const float* cos_row, const float* sin_row) {
+// The norm weights and the row's cos/sin of 32 head columns hc0 .. hc0 + 31
+// (loaded ahead of their use: the cos/sin rows come from L2)
+struct QkvTables {
+  uint4 w[4];
+  float4 c[4], s[4];
+};
+__device__ __forceinline__ void qkv_tables(QkvTables& t, int hc0, const uint16_t* w, const float* cos_row,
+                                           const float* sin_row) {
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
-    const int hc = hc0 + 8 * u;  // head column of the 8 values
-    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w + hc));
-    const float4 c4 = __ldg(reinterpret_cast<const float4*>(cos_row + hc / 2));
-    const float4 s4 = __ldg(reinterpret_cast<const float4*>(sin_row + hc / 2));
-    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-    const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+    const int hc = hc0 + 8 * u;
+    t.w[u] = __ldg(reinterpret_cast<const uint4*>(w + hc));
+    t.c[u] = __ldg(reinterpret_cast<const float4*>(cos_row + hc / 2));
+    t.s[u] = __ldg(reinterpret_cast<const float4*>(sin_row + hc / 2));
+  }
+}
+
+// Output of 32 columns of a Q or K head (in registers as fp32 layer outputs
+// y, with their tables): u = y * inv * w, then the rotary embedding of each
+// adjacent pair (2i, 2i+1) by the row's angle i, rounded to bf16 into 16-byte
+// units u0 .. u0 + 3 of the 128B-swizzled staging row.
+__device__ __forceinline__ void qkv_out32(uint8_t* buf, int lane, const float (&y)[32], int u0, float inv,
+                                          const QkvTables& t) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t ww[4] = {t.w[u].x, t.w[u].y, t.w[u].z, t.w[u].w};
+    const float cs[4] = {t.c[u].x, t.c[u].y, t.c[u].z, t.c[u].w}, sn[4] = {t.s[u].x, t.s[u].y, t.s[u].z, t.s[u].w};
     uint32_t w4[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -118,9 +135,6 @@ __device__ __forceinline__ void qkv_out32(uint8_t* buf, int lane, const float (&
     }
     *reinterpret_cast<uint4*>(buf + lane * 128 + (((u0 + u) ^ (lane & 7)) * 16)) =
         make_uint4(w4[0], w4[1], w4[2], w4[3]);
-    // one unit's table loads at a time (keeps them from being hoisted into
-    // registers that the caller's live values need)
-    asm volatile("" ::: "memory");
   }
 }
 
@@ -149,6 +163,16 @@ __device__ __forceinline__ void layer_out32(float (&y)[32], const uint32_t (&acc
 }
 
 
+// The column tile of tile sequence index t % tiles_n. With the fused QKV
+// epilogue and a whole number of tiles per Q/K/V section, the column tiles of
+// the three sections are interleaved (Q0, K0, V0, Q1, ...), so that the tiles
+// a CTA pair takes in turn mix the costly Q/K epilogues with plain V ones.
+__device__ __forceinline__ int column_tile(int t, int tiles_n, bool interleave) {
+  if (!interleave) return t;
+  const int per = tiles_n / 3;
+  return (t % 3) * per + t / 3;
+}
+
 // Epilogue of the instance: kEpiPlain (y = alpha acc + bias), kEpiQkv (the
 // fused QKV epilogue) or kEpiGelu (GELU of the layer output before its
 // rounding: the up-projection of the fused GELU-MLP). Separate instances, so
@@ -175,6 +199,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int nk = (p.K + BK - 1) / BK;
   const bool has_lr = p.r > 0;
+  // interleave the sections' column tiles when each section is whole tiles
+  const bool qkv_mix = kEpi == kEpiQkv && p.tiles_n % 3 == 0 && p.qkv_heads % 2 == 0 && p.qkv_heads / 2 * 3 == p.tiles_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -224,7 +250,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
       uint32_t it = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-        const int tm = tile / p.tiles_n, tn = tile % p.tiles_n;
+        const int tm = tile / p.tiles_n, tn = column_tile(tile % p.tiles_n, p.tiles_n, qkv_mix);
         const int row0 = tm * 256 + (int)rank * BM;      // this CTA's A rows
         const int col0 = tn * BN + (int)rank * (BN / 2);  // this CTA's B rows
         if (has_lr) {
@@ -348,7 +374,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     const int overlap_chunks = 64 / cols;          // chunks covering the 64 shared columns
     int i = 0;
     for (int tile = pair; tile < num_tiles; tile += npairs, ++i) {
-      const int tm = tile / p.tiles_n, tn = tile % p.tiles_n;
+      const int tm = tile / p.tiles_n, tn = column_tile(tile % p.tiles_n, p.tiles_n, qkv_mix);
       const int row0 = tm * 256 + (int)rank * BM + 32 * q;
       const int n0 = tn * BN + 128 * h;
       const int b = i & 1;
@@ -415,7 +441,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           // holds them) first: its layer outputs stay in registers; the other
           // chunk is read once for the sum of squares and again for the output
           float ya[32], yb[32];
-          float ss = 0.f;
+          // sum of squares in a fixed order, whatever the chunk order: per
+          // chunk even and odd columns in increasing order, then chunk 0 +
+          // chunk 1 (the result does not depend on the tile schedule)
+          float sf0 = 0.f, sf1 = 0.f, ss0 = 0.f, ss1 = 0.f;
           {
             uint32_t v[32];
             tmem_ld32(tbase + 64 * cf, v);
@@ -432,8 +461,19 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             }
             layer_out32(yb, v, alpha, p.bias, nh + 64 * cf + 32);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) ss = fmaf(yb[c], yb[c], fmaf(ya[c], ya[c], ss));
+            for (int c = 0; c < 32; c += 2) {
+              sf0 = fmaf(ya[c], ya[c], sf0);
+              sf1 = fmaf(ya[c + 1], ya[c + 1], sf1);
+            }
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              sf0 = fmaf(yb[c], yb[c], sf0);
+              sf1 = fmaf(yb[c + 1], yb[c + 1], sf1);
+            }
           }
+          // the first output slice's tables load under the sum-of-squares pass
+          QkvTables tab;
+          qkv_tables(tab, 64 * cf, wn, cos_row, sin_row);
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             uint32_t v16[16];
@@ -446,9 +486,11 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                   p.bias ? __ldg(reinterpret_cast<const uint32_t*>(p.bias + nh + 64 * cs + 16 * qq + c)) : 0u;
               const float t0 = fmaf(alpha, __uint_as_float(v16[c]), bf16_bits_to_f32(bw & 0xFFFFu));
               const float t1 = fmaf(alpha, __uint_as_float(v16[c + 1]), bf16_bits_to_f32(bw >> 16));
-              ss = fmaf(t1, t1, fmaf(t0, t0, ss));
+              ss0 = fmaf(t0, t0, ss0);
+              ss1 = fmaf(t1, t1, ss1);
             }
           }
+          const float ss = (sf0 + sf1) + (ss0 + ss1);  // addition commutes: chunk 0 + chunk 1
           const float inv = rsqrtf(fmaf(ss, 1.0f / 128.0f, p.eps));
 #pragma unroll 1
           for (int part = 0; part < 2; ++part) {
@@ -456,18 +498,20 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             __syncwarp();
             uint8_t* buf = sm.out[e][0];
             if (part == 0) {
-              qkv_out32(buf, lane, ya, 64 * cf, 0, inv, wn, cos_row, sin_row);
-              qkv_out32(buf, lane, yb, 64 * cf + 32, 4, inv, wn, cos_row, sin_row);
+              qkv_out32(buf, lane, ya, 0, inv, tab);
+              qkv_tables(tab, 64 * cf + 32, wn, cos_row, sin_row);
+              qkv_out32(buf, lane, yb, 4, inv, tab);
             } else {
 #pragma unroll 1
               for (int hh = 0; hh < 2; ++hh) {
+                qkv_tables(tab, 64 * cs + 32 * hh, wn, cos_row, sin_row);  // under the TMEM load
                 uint32_t v[32];
                 float t[32];
                 tmem_ld32(tbase + 64 * cs + 32 * hh, v);
                 tmem_ld_wait();
                 tmem_regs_ready(v);
                 layer_out32(t, v, alpha, p.bias, nh + 64 * cs + 32 * hh);
-                qkv_out32(buf, lane, t, 64 * cs + 32 * hh, 4 * hh, inv, wn, cos_row, sin_row);
+                qkv_out32(buf, lane, t, 4 * hh, inv, tab);
               }
             }
             fence_proxy_async_smem();

@@ -28,7 +28,7 @@ import torch
 __all__ = [
     "NVFP4", "INT4", "Status", "SvdqError", "PackedWeight", "QuantAct", "AwqWeight",
     "library_path", "load", "scale_bytes", "pack_weight", "quantize_act", "w4a4_linear",
-    "w4a4_linear_qkv", "qkv_norm_rope", "svdq_linear", "awq_pack_weight", "awq_w4a16_linear", "device_error", "set_wait_limit_ns",
+    "w4a4_linear_qkv", "qkv_norm_rope", "RopeTable", "pack_rope", "svdq_linear", "awq_pack_weight", "awq_w4a16_linear", "device_error", "set_wait_limit_ns",
     "probe_convert", "probe_wait_timeout", "probe_mma_peak", "debug_force_arch",
 ]
 
@@ -69,7 +69,9 @@ SIGNATURES = {
     "svdq_pack_weight": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P]),
     "svdq_quantize_act": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
-    "svdq_w4a4_linear_qkv": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P]),
+    "svdq_rope_packed_bytes": (C.c_size_t, [_I]),
+    "svdq_rope_pack": (_I, [_I, _P, _P, _P, _P]),
+    "svdq_w4a4_linear_qkv": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P]),
     "svdq_qkv_norm_rope": (_I, [_I, _I, _P, _P, _F, _P, _P, _P, _P]),
     "awq_pack_weight": (_I, [_I, _I, _P, _P, _P, _P, _P]),
     "awq_w4a16_linear": (_I, [_I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
@@ -296,12 +298,33 @@ def w4a4_linear(qa: QuantAct, pw: PackedWeight, bias: Optional[torch.Tensor] = N
     return out
 
 
+@dataclass
+class RopeTable:
+    """The rotary cos/sin tables of M rows in svdq_rope_pack's layout (fp32,
+    svdq_rope_packed_bytes(M) bytes)."""
+    M: int
+    data: torch.Tensor
+
+
+def pack_rope(cos: torch.Tensor, sin: torch.Tensor, stream=None) -> RopeTable:
+    """svdq_rope_pack: cos, sin fp32 [M, 64] -> the packed table the fused QKV
+    epilogue reads (once per set of positions; every layer can share it)."""
+    _need(cos.dim() == 2, "cos: expected [M, 64]")
+    M = cos.shape[0]
+    _is(cos, torch.float32, (M, 64), "cos")
+    _is(sin, torch.float32, (M, 64), "sin")
+    data = torch.empty(load().svdq_rope_packed_bytes(M) // 4, dtype=torch.float32, device=cos.device)
+    pc, ps, pr = _ptrs(cos, sin, data)
+    _check("svdq_rope_pack", load().svdq_rope_pack(M, pc, ps, pr, _stream(stream)))
+    return RopeTable(M, data)
+
+
 def w4a4_linear_qkv(qa: QuantAct, pw: PackedWeight, heads: int, norm_q: torch.Tensor, norm_k: torch.Tensor,
-                    eps: float, cos: torch.Tensor, sin: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                    eps: float, rope: RopeTable, bias: Optional[torch.Tensor] = None,
                     stream=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """svdq_w4a4_linear_qkv: the NVFP4 layer as a grouped Q/K/V projection (N =
     3 * heads * 128) with per-head RMSNorm of Q and K and the rotary embedding
-    in the GEMM's epilogue. cos, sin: fp32 [M, 64]."""
+    in the GEMM's epilogue. rope: pack_rope of the M rows' cos/sin [M, 64]."""
     M, K, N = qa.M, qa.K, pw.N
     _check_packed(pw)
     _need(pw.prec == NVFP4 and qa.prec == NVFP4, "the fused QKV epilogue is NVFP4 only")
@@ -314,8 +337,8 @@ def w4a4_linear_qkv(qa: QuantAct, pw: PackedWeight, heads: int, norm_q: torch.Te
         _is(qa.P, torch.bfloat16, (M, qa.r), "qa.P")
     _is(norm_q, torch.bfloat16, (128,), "norm_q")
     _is(norm_k, torch.bfloat16, (128,), "norm_k")
-    _is(cos, torch.float32, (M, 64), "cos")
-    _is(sin, torch.float32, (M, 64), "sin")
+    _need(isinstance(rope, RopeTable) and rope.M == M, "rope: expected pack_rope of the layer's {} rows", M)
+    _is(rope.data, torch.float32, (load().svdq_rope_packed_bytes(M) // 4,), "rope.data")
     if bias is not None:
         _is(bias, torch.bfloat16, (N,), "bias")
     if out is None:
@@ -323,8 +346,8 @@ def w4a4_linear_qkv(qa: QuantAct, pw: PackedWeight, heads: int, norm_q: torch.Te
     else:
         _is(out, torch.bfloat16, (M, N), "out")
     ptrs = _ptrs(qa.codes, qa.scales, qa.P, pw.codes, pw.scales, pw.tensor_scale, pw.lr_up, bias, norm_q, norm_k)
-    pc, ps, po = _ptrs(cos, sin, out)
-    _check("svdq_w4a4_linear_qkv", load().svdq_w4a4_linear_qkv(M, K, heads, pw.r, *ptrs, float(eps), pc, ps, po,
+    pr, po = _ptrs(rope.data, out)
+    _check("svdq_w4a4_linear_qkv", load().svdq_w4a4_linear_qkv(M, K, heads, pw.r, *ptrs, float(eps), pr, po,
                                                                _stream(stream)))
     return out
 

@@ -303,23 +303,42 @@ svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const
   return from_cuda(p == SVDQ_NVFP4 ? launch_gemm_nvfp4(a, s) : launch_gemm_int4(a, s));
 }
 
+size_t svdq_rope_packed_bytes(int M) {
+  if (M < 0) return 0;
+  return (size_t)((M + 31) / 32) * 16384;
+}
+
+svdq_status svdq_rope_pack(int M, const float* cos_t, const float* sin_t, float* rope, void* stream) {
+  if (M < 0) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!cos_t || !sin_t || !rope) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(cos_t) || !aligned16(sin_t) || !aligned16(rope)) return SVDQ_ERR_ALIGN;
+  const uintptr_t r0 = reinterpret_cast<uintptr_t>(rope), r1 = r0 + svdq_rope_packed_bytes(M);
+  for (const float* t : {cos_t, sin_t}) {
+    const uintptr_t t0 = reinterpret_cast<uintptr_t>(t), t1 = t0 + (size_t)M * 64 * sizeof(float);
+    if (r0 < t1 && t0 < r1) return SVDQ_ERR_INVALID_ARG;
+  }
+  svdq_status st = device_info(nullptr, nullptr);
+  if (st != SVDQ_OK) return st;
+  return from_cuda(launch_rope_pack(M, cos_t, sin_t, rope, static_cast<cudaStream_t>(stream)));
+}
+
 svdq_status svdq_w4a4_linear_qkv(int M, int K, int heads, int r, const uint8_t* x_codes, const void* x_scales,
                                  const uint16_t* P, const uint8_t* w_codes, const void* w_scales,
                                  const float* w_tensor_scale, const uint16_t* lr_up, const uint16_t* bias,
-                                 const uint16_t* norm_q, const uint16_t* norm_k, float eps, const float* cos_t,
-                                 const float* sin_t, uint16_t* y, void* stream) {
+                                 const uint16_t* norm_q, const uint16_t* norm_k, float eps, const float* rope,
+                                 uint16_t* y, void* stream) {
   svdq_status st = check_common(SVDQ_NVFP4, K, r);
   if (st != SVDQ_OK) return st;
   if (M < 0 || heads <= 0 || heads > (1 << 20) / 384) return SVDQ_ERR_INVALID_ARG;
   if (!(eps >= 0.0f && eps < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
-  if (!x_codes || !x_scales || !w_codes || !w_scales || !w_tensor_scale || !y || !norm_q || !norm_k || !cos_t ||
-      !sin_t)
+  if (!x_codes || !x_scales || !w_codes || !w_scales || !w_tensor_scale || !y || !norm_q || !norm_k || !rope)
     return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!P || !lr_up)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
       !aligned16(w_tensor_scale) || !aligned16(y) || !aligned16(norm_q) || !aligned16(norm_k) ||
-      !aligned16(cos_t) || !aligned16(sin_t) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3)) ||
+      !aligned16(rope) || (bias && (reinterpret_cast<uintptr_t>(bias) & 3)) ||
       (r > 0 && (!aligned16(P) || !aligned16(lr_up))))
     return SVDQ_ERR_ALIGN;
   unsigned* err = nullptr;
@@ -332,8 +351,7 @@ svdq_status svdq_w4a4_linear_qkv(int M, int K, int heads, int r, const uint8_t* 
   a.norm_q = norm_q;
   a.norm_k = norm_k;
   a.eps = eps;
-  a.cos_t = cos_t;
-  a.sin_t = sin_t;
+  a.rope = rope;
   return from_cuda(launch_gemm_nvfp4(a, static_cast<cudaStream_t>(stream)));
 }
 

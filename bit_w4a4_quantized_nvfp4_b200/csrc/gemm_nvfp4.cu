@@ -83,34 +83,35 @@ struct Params {
   unsigned* err;
   unsigned long long wait_ns;
   // fused QKV epilogue (qkv_heads > 0): N = 3 * qkv_heads * 128, Q, K, V in
-  // that order; RMSNorm weights [128] of Q and K heads, eps, rotary tables
-  // cos/sin fp32 [M, 64]
+  // that order; RMSNorm weights [128] of Q and K heads, eps, the rotary
+  // tables in the packed layout of svdq_rope_pack
   int qkv_heads;
   const uint16_t* norm_q;
   const uint16_t* norm_k;
   float eps;
-  const float* cos_t;
-  const float* sin_t;
+  const float* rope;
 };
 
 // Output of 32 columns of a Q or K head (head columns hc0 .. hc0 + 31, in
 // registers as fp32 layer outputs y): u = y * inv * w, then the rotary
 // embedding of each adjacent pair (2i, 2i+1) by the row's angle i, rounded to
 // bf16 into 16-byte units u0 .. u0 + 3 of the 128B-swizzled staging row.
-// The norm weights and the row's cos/sin of 32 head columns hc0 .. hc0 + 31
-// (loaded ahead of their use: the cos/sin rows come from L2)
+// The norm weights and the lane's row's cos/sin of 32 head columns hc0 ..
+// hc0 + 31 (loaded ahead of their use: the tables come from L2). rope_lane
+// points at the lane's row in its 32-row block of the packed table: a group
+// of 4 rotary pairs (8 head columns) is a cos part and a sin part of
+// [32 rows][4], so the warp's 32 rows read 512 contiguous bytes per load.
 struct QkvTables {
   uint4 w[4];
   float4 c[4], s[4];
 };
-__device__ __forceinline__ void qkv_tables(QkvTables& t, int hc0, const uint16_t* w, const float* cos_row,
-                                           const float* sin_row) {
+__device__ __forceinline__ void qkv_tables(QkvTables& t, int hc0, const uint16_t* w, const float* rope_lane) {
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int hc = hc0 + 8 * u;
     t.w[u] = __ldg(reinterpret_cast<const uint4*>(w + hc));
-    t.c[u] = __ldg(reinterpret_cast<const float4*>(cos_row + hc / 2));
-    t.s[u] = __ldg(reinterpret_cast<const float4*>(sin_row + hc / 2));
+    t.c[u] = __ldg(reinterpret_cast<const float4*>(rope_lane + (hc / 8) * 256));
+    t.s[u] = __ldg(reinterpret_cast<const float4*>(rope_lane + (hc / 8) * 256 + 128));
   }
 }
 
@@ -433,10 +434,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         {
           const uint16_t* wn = sect == 0 ? p.norm_q : p.norm_k;
           const int nh = head * 128;
-          const int m = row0 + lane;
-          const int mc = m < p.M ? m : p.M - 1;  // a row past M is not stored: read any valid one
-          const float* cos_row = p.cos_t + (size_t)mc * 64;
-          const float* sin_row = p.sin_t + (size_t)mc * 64;
+          // the warp's 32 rows are one block of the packed table (a quadrant
+          // wholly past M reads the last block: its rows are not stored)
+          const int blk = (row0 < p.M ? row0 : p.M - 1) / 32;
+          const float* rope_lane = p.rope + (size_t)blk * 4096 + 4 * lane;
           // the 64-column chunk that holds the shared columns (when this warp
           // holds them) first: its layer outputs stay in registers; the other
           // chunk is read once for the sum of squares and again for the output
@@ -473,7 +474,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
           }
           // the first output slice's tables load under the sum-of-squares pass
           QkvTables tab;
-          qkv_tables(tab, 64 * cf, wn, cos_row, sin_row);
+          qkv_tables(tab, 64 * cf, wn, rope_lane);
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             uint32_t v16[16];
@@ -499,12 +500,12 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             uint8_t* buf = sm.out[e][0];
             if (part == 0) {
               qkv_out32(buf, lane, ya, 0, inv, tab);
-              qkv_tables(tab, 64 * cf + 32, wn, cos_row, sin_row);
+              qkv_tables(tab, 64 * cf + 32, wn, rope_lane);
               qkv_out32(buf, lane, yb, 4, inv, tab);
             } else {
 #pragma unroll 1
               for (int hh = 0; hh < 2; ++hh) {
-                qkv_tables(tab, 64 * cs + 32 * hh, wn, cos_row, sin_row);  // under the TMEM load
+                qkv_tables(tab, 64 * cs + 32 * hh, wn, rope_lane);  // under the TMEM load
                 uint32_t v[32];
                 float t[32];
                 tmem_ld32(tbase + 64 * cs + 32 * hh, v);
@@ -654,8 +655,7 @@ cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s) {
   p.norm_q = a.norm_q;
   p.norm_k = a.norm_k;
   p.eps = a.eps;
-  p.cos_t = a.cos_t;
-  p.sin_t = a.sin_t;
+  p.rope = a.rope;
 
   const size_t smem = sizeof(Smem) + 1024;
   auto kern = p.qkv_heads > 0 ? gemm_nvfp4_kernel<kEpiQkv>

@@ -85,8 +85,7 @@ struct GemmArgs {
   const uint16_t* norm_q = nullptr;
   const uint16_t* norm_k = nullptr;
   float eps = 0.f;
-  const float* cos_t = nullptr;
-  const float* sin_t = nullptr;
+  const float* rope = nullptr;  // cos/sin packed by svdq_rope_pack
 };
 cudaError_t launch_gemm_nvfp4(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_int4(const GemmArgs& a, cudaStream_t s);
@@ -101,6 +100,9 @@ struct NormRopeArgs {
   float eps;
 };
 cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s);
+
+// cos/sin [M, 64] -> the packed rotary table (16384 * ceil(M / 32) bytes)
+cudaError_t launch_rope_pack(int M, const float* cos_t, const float* sin_t, float* rope, cudaStream_t s);
 
 cudaError_t launch_probe_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3,
                                  uint16_t* bf16, cudaStream_t s);

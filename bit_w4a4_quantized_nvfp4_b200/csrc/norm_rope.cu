@@ -10,6 +10,9 @@
 // weights once, then takes the heads warp, warp + 8, ... (all their loads in
 // flight at once). The sum of squares is a warp-shuffle reduction. Bound by
 // HBM: the Q and K sections are read and written once.
+//
+// Also here: the pack of the cos/sin tables into the 32-row-block layout that
+// the fused epilogue reads (svdq_rope_pack).
 #include "device.cuh"
 #include "kernels.h"
 
@@ -58,10 +61,32 @@ norm_rope_kernel(NormRopeArgs a) {
   }
 }
 
+// The packed rotary table: one CTA per 32-row block, thread (row lane,
+// group g) moves the cos and sin of pairs 4g .. 4g + 3 of its row (zero for
+// rows past M). The writes of a group are 512 contiguous bytes per table.
+__global__ void __launch_bounds__(512) rope_pack_kernel(int M, const float* __restrict__ cos_t,
+                                                        const float* __restrict__ sin_t, float* __restrict__ rope) {
+  const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int blk = blockIdx.x, m = blk * 32 + lane;
+  float4 c = make_float4(0.f, 0.f, 0.f, 0.f), sn = c;
+  if (m < M) {
+    c = __ldg(reinterpret_cast<const float4*>(cos_t + (size_t)m * 64 + 4 * g));
+    sn = __ldg(reinterpret_cast<const float4*>(sin_t + (size_t)m * 64 + 4 * g));
+  }
+  float* dst = rope + ((size_t)blk * 16 + g) * 256 + 4 * lane;
+  *reinterpret_cast<float4*>(dst) = c;
+  *reinterpret_cast<float4*>(dst + 128) = sn;
+}
+
 }  // namespace
 
 cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s) {
   norm_rope_kernel<<<(unsigned)a.M, kWarpsNR * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_pack(int M, const float* cos_t, const float* sin_t, float* rope, cudaStream_t s) {
+  rope_pack_kernel<<<(unsigned)((M + 31) / 32), 512, 0, s>>>(M, cos_t, sin_t, rope);
   return cudaGetLastError();
 }
 

@@ -156,6 +156,28 @@ svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const
                              const uint16_t* lr_up, const uint16_t* bias, void* y,
                              svdq_out_dtype out, void* stream);
 
+/* svdq_rope_packed_bytes — bytes of the packed rotary table that
+ * svdq_rope_pack writes for M rows: 16384 * ceil(M / 32). 0 for M < 0. */
+size_t svdq_rope_packed_bytes(int M);
+
+/* svdq_rope_pack — the rotary embedding's cos/sin tables in the layout the
+ * fused QKV epilogue reads (a change of layout only: no arithmetic and no
+ * step of the method itself). The tables depend only on the tokens' positions, so one
+ * pack serves every attention layer of a forward pass.
+ * In:  cos_t, sin_t fp32 [M, 64] (row m = the token's angles for the rotary
+ *      pairs i = 0..63).
+ * Out: rope fp32, svdq_rope_packed_bytes(M) bytes: blocks of 32 rows, each
+ *      block 16 groups of 4 pairs, each group the cos part then the sin part,
+ *      each part [32 rows][4 pairs]:
+ *        cos[m, i] at float offset ((m/32 * 16 + i/4) * 2 + 0) * 128 + (m%32) * 4 + i%4
+ *        sin[m, i] at the same offset + 128.
+ *      Rows past M in the last block are written as zero.
+ *      A warp whose lanes hold 32 consecutive rows reads one group of a table
+ *      as 512 contiguous bytes (the plain [M, 64] rows would be 32 strided
+ *      pieces).
+ * Pointers 16-byte aligned; rope must not overlap cos_t or sin_t. */
+svdq_status svdq_rope_pack(int M, const float* cos_t, const float* sin_t, float* rope, void* stream);
+
 /* svdq_w4a4_linear_qkv — the NVFP4 layer as a grouped Q/K/V projection with
  * the per-head RMSNorm of Q and K and the rotary embedding fused into the
  * GEMM's epilogue (Diffusers "Nunchaku Lite" page, section on fused kernels:
@@ -168,22 +190,23 @@ svdq_status svdq_w4a4_linear(svdq_precision p, int M, int K, int N, int r, const
  *     y[2i] = u[2i] cos[m,i] - u[2i+1] sin[m,i]; y[2i+1] = u[2i] sin[m,i] + u[2i+1] cos[m,i]
  *   V heads: y = y_l. Output rounded to bf16 once.
  * In:  as svdq_w4a4_linear (NVFP4); heads = heads per section (head_dim 128,
- *      N = 3 * heads * 128); norm_q, norm_k bf16 [128]; eps >= 0; cos_t,
- *      sin_t fp32 [M, 64] (row m = the token's angles for pairs i = 0..63).
+ *      N = 3 * heads * 128); norm_q, norm_k bf16 [128]; eps >= 0; rope = the
+ *      M rows' cos/sin tables packed by svdq_rope_pack (for the same M).
  * Out: y bf16 [M, N].
  * Pointers 16-byte aligned (bias 4-byte). */
 svdq_status svdq_w4a4_linear_qkv(int M, int K, int heads, int r, const uint8_t* x_codes, const void* x_scales,
                                  const uint16_t* P, const uint8_t* w_codes, const void* w_scales,
                                  const float* w_tensor_scale, const uint16_t* lr_up, const uint16_t* bias,
-                                 const uint16_t* norm_q, const uint16_t* norm_k, float eps, const float* cos_t,
-                                 const float* sin_t, uint16_t* y, void* stream);
+                                 const uint16_t* norm_q, const uint16_t* norm_k, float eps, const float* rope,
+                                 uint16_t* y, void* stream);
 
 /* svdq_qkv_norm_rope — the same per-head RMSNorm and rotary embedding as
  * svdq_w4a4_linear_qkv, as a separate pass over a grouped Q/K/V projection's
  * bf16 output y [M, 3 * heads * 128] (Q and K sections updated in place, V
  * untouched). It reads the rounded output, so it is the unfused form of the
  * operator that svdq_w4a4_linear_qkv computes on the unrounded accumulator.
- * Arguments as svdq_w4a4_linear_qkv; pointers 16-byte aligned. */
+ * Arguments as svdq_w4a4_linear_qkv, but with the plain tables: cos_t, sin_t
+ * fp32 [M, 64]; pointers 16-byte aligned. */
 svdq_status svdq_qkv_norm_rope(int M, int heads, const uint16_t* norm_q, const uint16_t* norm_k, float eps,
                                const float* cos_t, const float* sin_t, uint16_t* y, void* stream);
 

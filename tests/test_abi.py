@@ -211,13 +211,13 @@ def test_binding_checks_pack_and_awq(lib):
 def test_qkv_entry_validation(lib):
     S = svdq.Status
     f = lib.svdq_w4a4_linear_qkv
-    # (M, K, heads, r, x_codes, x_scales, P, w_codes, w_scales, ts, lr_up, bias, nq, nk, eps, cos, sin, y, stream)
-    ok = [4, 64, 1, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1e-6, FAKE, FAKE, FAKE, None]
+    # (M, K, heads, r, x_codes, x_scales, P, w_codes, w_scales, ts, lr_up, bias, nq, nk, eps, rope, y, stream)
+    ok = [4, 64, 1, 0, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, 1e-6, FAKE, FAKE, None]
 
     def call(**kw):
         args = list(ok)
-        names = ["M", "K", "heads", "r", "xc", "xs", "P", "wc", "ws", "ts", "lr", "b", "nq", "nk", "eps", "cos",
-                 "sin", "y", "s"]
+        names = ["M", "K", "heads", "r", "xc", "xs", "P", "wc", "ws", "ts", "lr", "b", "nq", "nk", "eps", "rope",
+                 "y", "s"]
         for k, v in kw.items():
             args[names.index(k)] = v
         return f(*args)
@@ -226,20 +226,38 @@ def test_qkv_entry_validation(lib):
     assert call(K=96) == S.SHAPE
     assert call(eps=-1.0) == S.INVALID_ARG
     assert call(nq=None) == S.INVALID_ARG
-    assert call(cos=None) == S.INVALID_ARG
+    assert call(rope=None) == S.INVALID_ARG
     assert call(r=16) == S.INVALID_ARG            # r > 0 needs P and lr_up
-    assert call(sin=FAKE + 4) == S.ALIGN
-    assert call(M=0, xc=None, xs=None, wc=None, ws=None, ts=None, nq=None, nk=None, cos=None, sin=None,
-                y=None) == S.OK
+    assert call(rope=FAKE + 4) == S.ALIGN
+    assert call(M=0, xc=None, xs=None, wc=None, ws=None, ts=None, nq=None, nk=None, rope=None, y=None) == S.OK
+
+
+def test_rope_pack_entry_validation(lib):
+    S = svdq.Status
+    f = lib.svdq_rope_pack
+    assert lib.svdq_rope_packed_bytes(0) == 0
+    assert lib.svdq_rope_packed_bytes(1) == 16384
+    assert lib.svdq_rope_packed_bytes(64) == 2 * 16384
+    assert lib.svdq_rope_packed_bytes(65) == 3 * 16384
+    assert lib.svdq_rope_packed_bytes(-1) == 0
+    far = FAKE + (1 << 24)
+    assert f(-1, FAKE, FAKE + 65536, far, None) == S.INVALID_ARG
+    assert f(0, None, None, None, None) == S.OK
+    assert f(4, None, FAKE + 65536, far, None) == S.INVALID_ARG
+    assert f(4, FAKE + 8, FAKE + 65536, far, None) == S.ALIGN
+    assert f(4, FAKE, FAKE + 65536, FAKE + 512, None) == S.INVALID_ARG   # rope overlaps cos
 
 
 def test_binding_checks_qkv(lib):
     pw, qa = _packed(N=384), _act()
     nq, nk = _bf16(128), _bf16(128)
-    cs, sn = torch.zeros(8, 64), torch.zeros(8, 64)
-    _raises("CUDA", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, cs, sn)   # well formed
-    _raises("3 \\* heads", svdq.w4a4_linear_qkv, qa, pw, 2, nq, nk, 1e-6, cs, sn)
-    _raises("norm_q: shape", svdq.w4a4_linear_qkv, qa, pw, 1, _bf16(64), nk, 1e-6, cs, sn)
-    _raises("cos: shape", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, torch.zeros(8, 32), sn)
+    rope = svdq.RopeTable(8, torch.zeros(4096))
+    _raises("CUDA", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, rope)   # well formed
+    _raises("3 \\* heads", svdq.w4a4_linear_qkv, qa, pw, 2, nq, nk, 1e-6, rope)
+    _raises("norm_q: shape", svdq.w4a4_linear_qkv, qa, pw, 1, _bf16(64), nk, 1e-6, rope)
+    _raises("rope: expected", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, svdq.RopeTable(9, torch.zeros(4096)))
+    _raises("rope.data: shape", svdq.w4a4_linear_qkv, qa, pw, 1, nq, nk, 1e-6, svdq.RopeTable(8, torch.zeros(64)))
     _raises("NVFP4 only", svdq.w4a4_linear_qkv, _act(prec=svdq.INT4), _packed(prec=svdq.INT4, N=384), 1, nq, nk,
-            1e-6, cs, sn)
+            1e-6, rope)
+    _raises("cos: shape", svdq.pack_rope, torch.zeros(8, 32), torch.zeros(8, 64))
+    _raises("sin: dtype", svdq.pack_rope, torch.zeros(8, 64), torch.zeros(8, 64, dtype=torch.float64))

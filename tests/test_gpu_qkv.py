@@ -44,7 +44,8 @@ def run_case(d, e, heads, rows=None, bias=True):
     qa = svdq.quantize_act(bf16_dev(d["x"]), pw, L1)
     b = bf16_dev(d["b"]) if bias else None
     cos, sin = torch.from_numpy(e["cos"]).cuda(), torch.from_numpy(e["sin"]).cuda()
-    y = svdq.w4a4_linear_qkv(qa, pw, heads, bf16_dev(e["wq"]), bf16_dev(e["wk"]), e["eps"], cos, sin, b)
+    rope = svdq.pack_rope(cos, sin)
+    y = svdq.w4a4_linear_qkv(qa, pw, heads, bf16_dev(e["wq"]), bf16_dev(e["wk"]), e["eps"], rope, b)
     y_plain = svdq.w4a4_linear(qa, pw, b)
     torch.cuda.synchronize()
     assert svdq.device_error() == 0
@@ -72,7 +73,7 @@ def test_qkv_epilogue_matches_oracle(M, K, heads, r, bias):
 
 def test_qkv_epilogue_c3_full_size():
     """The fused-QKV projection of the benchmark workload (M4608 K3072, 24
-    heads of 128 per section, N 9216, r 32) with the C3 rotary tables: 128
+    heads of 128 per section, N 9216, r 32) with the C3 rotary tables: 512
     seeded rows against the oracle, the V section against the plain layer."""
     c = synth.CONFIGS["c3_qkv_nvfp4"]
     d = synth.config_layer("c3_qkv_nvfp4")
@@ -98,3 +99,22 @@ def test_separate_norm_rope_pass_matches_oracle(M, heads):
     yo = oracle.qkv_norm_rope(oracle.bf16_to_f32(yb).astype(np.float64), heads, 128, e["wq"], e["wk"], e["eps"],
                               e["cos"], e["sin"])
     check_bf16_output(oracle.bf16_to_f32(yg), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))
+
+
+@pytest.mark.parametrize("M", [77, 64, 1])
+def test_rope_pack_layout(M):
+    """svdq_rope_pack moves every cos/sin value, unchanged, to the offset the
+    header states; the rows that pad the last 32-row block are zero."""
+    e = synth.qkv_epilogue_inputs(44, M, 128, 1)
+    rope = svdq.pack_rope(torch.from_numpy(e["cos"]).cuda(), torch.from_numpy(e["sin"]).cuda())
+    torch.cuda.synchronize()
+    got = rope.data.cpu().numpy().view(np.uint32)
+    nb = (M + 31) // 32
+    assert got.size == nb * 4096
+    want = np.zeros(nb * 4096, np.uint32)
+    for tab, part in ((e["cos"], 0), (e["sin"], 1)):
+        bits = np.ascontiguousarray(tab, np.float32).view(np.uint32)
+        for m in range(M):
+            for i in range(64):
+                want[((m // 32 * 16 + i // 4) * 2 + part) * 128 + (m % 32) * 4 + i % 4] = bits[m, i]
+    assert np.array_equal(got, want)

@@ -501,7 +501,7 @@ def bench_mlp(svdq, flush, steps=30):
         svdq.w4a4_linear(qa_d, pw_d, bd, out=y)
 
     res = {}
-    for name, fn in (("fused_ms", fused), ("unfused_ms", unfused), ("rope_pack_ms", pack)):
+    for name, fn in (("fused_ms", fused), ("unfused_ms", unfused)):
         ts = []
         for i in range(steps + 3):
             flush.zero_()

@@ -118,3 +118,30 @@ def test_rope_pack_layout(M):
             for i in range(64):
                 want[((m // 32 * 16 + i // 4) * 2 + part) * 128 + (m % 32) * 4 + i % 4] = bits[m, i]
     assert np.array_equal(got, want)
+
+
+def test_qkv_epilogue_writes_nothing_past_y():
+    """The fused epilogue's output lives in a larger buffer filled with a
+    sentinel: after the call the bytes past y still hold it (ragged M, an odd
+    head count so the last column tile is half past N), and y matches the
+    oracle."""
+    M, K, heads, r = 77, 256, 3, 16
+    N = 3 * heads * 128
+    d = synth.svdq_layer(45, M, K, N, r)
+    e = synth.qkv_epilogue_inputs(45, M, 128, heads)
+    L1, L2 = bf16_dev(d["L1"]), bf16_dev(d["L2"])
+    pw = svdq.pack_weight("nvfp4", torch.from_numpy(d["W"]).cuda(), torch.from_numpy(d["lam"]).cuda(), L1, L2)
+    qa = svdq.quantize_act(bf16_dev(d["x"]), pw, L1)
+    rope = svdq.pack_rope(torch.from_numpy(e["cos"]).cuda(), torch.from_numpy(e["sin"]).cuda())
+    pad = 8192
+    buf = torch.full((M * N + pad,), -555.0, dtype=torch.bfloat16, device="cuda")
+    y = buf[: M * N].view(M, N)
+    svdq.w4a4_linear_qkv(qa, pw, heads, bf16_dev(e["wq"]), bf16_dev(e["wk"]), e["eps"], rope, bf16_dev(d["b"]), out=y)
+    torch.cuda.synchronize()
+    assert svdq.device_error() == 0
+    assert (buf[M * N:] == -555.0).all(), "write past the end of y"
+    w = oracle.pack_weight("nvfp4", d["W"], d["lam"], d["L1"], d["L2"])
+    a = oracle.quantize_act("nvfp4", d["x"], w["inv_lam"], 1.0, d["L1"])
+    yl = oracle.linear("nvfp4", a, w, 1.0, d["L2"], d["b"])
+    yo = oracle.qkv_norm_rope(yl, heads, 128, e["wq"], e["wk"], e["eps"], e["cos"], e["sin"])
+    check_bf16_output(oracle.bf16_to_f32(bf16_np(y)), yo, oracle.bf16_to_f32(oracle.bf16_rn(yo)))

@@ -162,8 +162,8 @@ size_t svdq_rope_packed_bytes(int M);
 
 /* svdq_rope_pack — the rotary embedding's cos/sin tables in the layout the
  * fused QKV epilogue reads (a change of layout only: no arithmetic and no
- * step of the method itself). The tables depend only on the tokens' positions, so one
- * pack serves every attention layer of a forward pass.
+ * step of the method itself). The tables depend only on the tokens'
+ * positions, so one pack serves every attention layer of a forward pass.
  * In:  cos_t, sin_t fp32 [M, 64] (row m = the token's angles for the rotary
  *      pairs i = 0..63).
  * Out: rope fp32, svdq_rope_packed_bytes(M) bytes: blocks of 32 rows, each
@@ -175,7 +175,9 @@ size_t svdq_rope_packed_bytes(int M);
  *      A warp whose lanes hold 32 consecutive rows reads one group of a table
  *      as 512 contiguous bytes (the plain [M, 64] rows would be 32 strided
  *      pieces).
- * Pointers 16-byte aligned; rope must not overlap cos_t or sin_t. */
+ * The caller allocates rope. Pointers 16-byte aligned (else SVDQ_ERR_ALIGN);
+ * M < 0, a NULL pointer, or rope overlapping cos_t or sin_t give
+ * SVDQ_ERR_INVALID_ARG; M = 0 is a no-op. */
 svdq_status svdq_rope_pack(int M, const float* cos_t, const float* sin_t, float* rope, void* stream);
 
 /* svdq_w4a4_linear_qkv — the NVFP4 layer as a grouped Q/K/V projection with

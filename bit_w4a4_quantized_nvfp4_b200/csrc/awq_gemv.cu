@@ -32,7 +32,10 @@
 // 64 x 256-K boxes, 128-byte swizzle, 16 KB) through a 4-stage TMA ring with
 // full/empty mbarriers; two warp groups (stage phases) take alternate stages,
 // four row tiles of 16 rows each; the CTA's activations, scales and zero
-// points are bulk-copied into shared memory once. With programmatic dependent
+// points are bulk-copied into shared memory once, the activations on one
+// barrier and the scales and zero points on another, so that the activation
+// conversion starts as soon as x has landed and the scales are waited for
+// only before a group's result is first scaled. With programmatic dependent
 // launch the CTA's first weight stages and its scales and zero points are
 // prefetched into L2 before the wait for the previous kernel in the stream (a
 // prefetch only moves data closer, L2 being the point of coherence) and
@@ -121,7 +124,7 @@ struct GemvLayout {
     off_z = off_s + ((kRowsG * sz_pitch + 15) / 16) * 16;
     off_red = off_z + ((kRowsG * sz_pitch + 15) / 16) * 16;
     off_bar = off_red + (kPhasesG - 1) * 4 * 32 * 2 * 4;
-    total = off_bar + 2 * kStagesG * 8 + 8 + 8;
+    total = off_bar + 2 * kStagesG * 8 + 8 + 8 + 8;
   }
 };
 
@@ -148,7 +151,8 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
   uint64_t* full = reinterpret_cast<uint64_t*>(base + L.off_bar);
   uint64_t* empty = full + kStagesG;
   uint64_t* xbar = empty + kStagesG;
-  int* abort_flag = reinterpret_cast<int*>(xbar + 1);
+  uint64_t* szbar = xbar + 1;
+  int* abort_flag = reinterpret_cast<int*>(szbar + 1);
   const uint32_t sz_bytes = (uint32_t)(min(kRowsG, N - n0) * L.sz_pitch);
 
   if (threadIdx.x == 0) launch_dependents();
@@ -158,6 +162,7 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
       mbar_init(&empty[s], 4);
     }
     mbar_init(xbar, 1);
+    mbar_init(szbar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -188,10 +193,11 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
         tma_load_2d(dst, &tm_q, &full[s], cc * (kStageKG / 2), n0);
         tma_load_2d(dst + kBoxBytesG, &tm_q, &full[s], cc * (kStageKG / 2) + 128, n0);
       };
-      mbar_expect_tx(xbar, (uint32_t)(M * 2 * K) + 2 * sz_bytes);
+      mbar_expect_tx(xbar, (uint32_t)(M * 2 * K));
       for (int m = 0; m < M; ++m) bulk_load(xs + m * L.x_pitch, a.x + (size_t)m * K, (uint32_t)(2 * K), xbar);
-      bulk_load(base + L.off_s, a.s + (size_t)n0 * ng, sz_bytes, xbar);
-      bulk_load(base + L.off_z, a.z + (size_t)n0 * ng, sz_bytes, xbar);
+      mbar_expect_tx(szbar, 2 * sz_bytes);
+      bulk_load(base + L.off_s, a.s + (size_t)n0 * ng, sz_bytes, szbar);
+      bulk_load(base + L.off_z, a.z + (size_t)n0 * ng, sz_bytes, szbar);
       for (; c < nst && c < kStagesG; ++c) issue_stage(c);
       for (int cc = kStagesG; cc < nst; ++cc) {
         tma_prefetch_l2_2d(&tm_q, cc * (kStageKG / 2), n0);
@@ -207,6 +213,7 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
       }
       // let the copies already issued land before the CTA can exit (bounded)
       (void)mbar_wait(xbar, 0, wait_ns, ok ? err : nullptr);
+      (void)mbar_wait(szbar, 0, wait_ns, ok ? err : nullptr);
       if (!ok)
         for (int j = max(0, c - kStagesG); j < c; ++j)
           (void)mbar_wait(&full[j % kStagesG], (j / kStagesG) & 1, wait_ns, nullptr);
@@ -307,6 +314,7 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
     return *reinterpret_cast<const uint4*>(box + r * 128 + ((ch ^ (r & 7)) << 4));
   };
 
+  bool sz_ready = false;
   for (int c = kh; c < nst && ok; c += kPhasesG) {
     const int s = c % kStagesG;
     if (!warp_wait(&full[s], (c / kStagesG) & 1, wait_ns, err)) {
@@ -354,6 +362,10 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
 #pragma unroll
       for (int e = 0; e < 4; ++e) cc[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
       keep = cc[0] + cc[1] + cc[2] + cc[3];
+      if (!sz_ready) {
+        if (!warp_wait(szbar, 0, wait_ns, err)) { ok = false; break; }
+        sz_ready = true;
+      }
       finish(cc, g0);
     } else {
       // blocks of G groups (8 / G per stage, each inside one box). Lane
@@ -396,6 +408,10 @@ awq_gemv_kernel(const __grid_constant__ CUtensorMap tm_q, AwqArgs a, unsigned* e
 #pragma unroll
         for (int e = 0; e < 4; ++e) cc[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
         keep += cc[0] + cc[1] + cc[2] + cc[3];
+        if (!sz_ready) {
+          if (!warp_wait(szbar, 0, wait_ns, err)) { ok = false; break; }
+          sz_ready = true;
+        }
         finish(cc, gb0);
       }
     }

@@ -226,15 +226,18 @@ quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     for (int c = 0; c < nchunks && c < 2; ++c)
       for (int b = 0; b < min(kChunk, K - c * kChunk) / 64; ++b) tma_prefetch_l2_2d(&tm_x, c * kChunk + 64 * b, row0);
   }
+  __syncthreads();  // the barriers are initialised
   // every input may be the previous kernel's output, every output may still
   // be read by it
   grid_dependency_wait();
-  const float s_tx = PREC == 0 ? a.tensor_scale[1] : 1.0f;
+  // the producer starts its loads at once; the consumers first tabulate the
+  // scale steps (named barrier 1: consumer warps only)
+  const float s_tx = PREC == 0 && warp < CW ? a.tensor_scale[1] : 1.0f;
   if (PREC == 0 && threadIdx.x < 256) {
     const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), s_tx);
     rtab[threadIdx.x] = d != 0.f ? make_float2(__frcp_rn(d), 0.f) : make_float2(0.f, 1.f);
   }
-  __syncthreads();
+  if (warp < CW) named_sync(1, CW * 32);
 
   if (warp == CW) {
     // ------------------------------------------------------------ producer

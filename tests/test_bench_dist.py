@@ -72,3 +72,13 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
 
     assert bench.run_reference(Args()) is None
     assert capsys.readouterr().out == ""
+
+
+def test_trimmed_mean_drops_both_tails():
+    import bench
+
+    xs = [1.0] * 8 + [100.0, -50.0]
+    assert bench.trimmed_mean(xs, 0.1) == 1.0
+    assert bench.trimmed_mean([2.0, 4.0], 0.1) == 3.0          # too few samples to trim
+    ticks = [89.088] * 6 + [90.112] * 4                         # event times on a 1.024 us grid
+    assert abs(bench.trimmed_mean(ticks, 0.1) - (5 * 89.088 + 3 * 90.112) / 8) < 1e-9
